@@ -1,0 +1,456 @@
+"""Benchmark of the low-bit matmul library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch of seeded synthetic input: for every shape
+of the workload one matmul call (argument checks, configuration lookup, split-K zeroing when
+the configuration splits K, the kernel). The per-shape configuration search runs once before
+the timed region, as a deployment would run it once per shape. Inputs sit in HBM before the
+timed region; weight sets rotate so that no call finds its weights in L2.
+
+Prints one JSON line (rank 0). Under torchrun every rank runs the same workload on its own GPU
+(independent replicas, no collective on the data path); `value` is the whole-job throughput
+(all ranks' FLOPs over the slowest rank's time).
+
+--impl reference times the host oracle (plain C, fp64) on a bounded sample of the same
+workload on this machine's cores and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+
+# ---- workloads -------------------------------------------------------------------------------
+# Each shape: (M, K, N). W4A16: group_size 128, fp16 zeros fixed at 8 (has_zero=1) unless noted.
+WORKLOADS = {
+    # int4-weight GEMM sweep over M at N = K = 16384 (the BitBLAS Matmul benchmark shapes)
+    "w4a16_nk16384": {"op": "w4a16", "has_zero": 1,
+                      "shapes": [(1, 16384, 16384), (32, 16384, 16384), (128, 16384, 16384),
+                                 (512, 16384, 16384), (16384, 16384, 16384)]},
+    # LLaMA-style layer shapes (hidet issue #364, k-parts=4 table), M = 1 and 128
+    "w4a16_llama": {"op": "w4a16", "has_zero": 1,
+                    "shapes": [(1, 4096, 11008), (1, 11008, 4096), (1, 4096, 4096),
+                               (1, 4096, 32000), (128, 4096, 11008), (128, 11008, 4096),
+                               (128, 4096, 4096), (128, 4096, 32000)]},
+    # the small-M part of the sweep alone
+    "w4a16_nk16384_small_m": {"op": "w4a16", "has_zero": 1,
+                              "shapes": [(1, 16384, 16384), (32, 16384, 16384),
+                                         (128, 16384, 16384)]},
+}
+DEFAULT_WORKLOAD = "w4a16_llama"
+
+
+def shape_bytes(op, M, K, N, has_zero, gs=128):
+    if op == "w4a16":
+        return N * K // 2 + N * (K // gs) * 2 * (1 + has_zero) + 2 * M * K + 2 * M * N
+    if op == "w8a8":
+        return N * K + M * K + 4 * M * N
+    if op == "w2a8":
+        return N * K // 4 + M * K + 4 * M * N
+    return 2 * N * K + 2 * M * K + 2 * M * N
+
+
+def shape_flops(M, K, N):
+    return 2.0 * M * N * K
+
+
+# ---- helpers ------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qgemm_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---- our arm ----------------------------------------------------------------------------------------
+
+def run_ours(args, world, rank, local):
+    import torch
+    import gemv_w4a16_w8a8_b200 as qg
+    from gemv_w4a16_w8a8_b200 import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    wl = WORKLOADS[args.workload]
+    op, hz, gs = wl["op"], wl["has_zero"], 128
+    shapes = wl["shapes"]
+    peaks = load_peaks()
+
+    # inputs: one A per shape; weights: one packed set per shape, replicated so that a step
+    # never reads weights that an earlier step left in L2
+    step_w_bytes = sum(N * K // 2 for _, K, N in shapes)
+    n_sets = max(1, math.ceil(3 * L2_BYTES / step_w_bytes))
+    n_sets = min(n_sets, 8)
+    per_shape = []
+    for si, (M, K, N) in enumerate(shapes):
+        d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=1000 * si)
+        A = torch.from_numpy(d["A"]).to(dev)
+        codes = torch.from_numpy(d["codes"]).to(dev)
+        S = torch.from_numpy(d["scales"]).to(dev)
+        Z = torch.from_numpy(d["zeros"]).to(dev) if hz else None
+        Wq0 = qg.quant_pack_int4(codes)
+        del codes
+        sets = [Wq0] + [Wq0.clone() for _ in range(n_sets - 1)]
+        C = torch.empty((M, N), dtype=torch.float16, device=dev)
+        per_shape.append({"M": M, "K": K, "N": N, "A": A, "S": S, "Z": Z, "W": sets, "C": C,
+                          "A_host": torch.from_numpy(d["A"]).pin_memory(),
+                          "C_host": torch.empty((M, N), dtype=torch.float16).pin_memory()})
+        del d
+    torch.cuda.synchronize()
+
+    # configuration search (once per shape, before timing)
+    tuned = []
+    for sp in per_shape:
+        M, K, N = sp["M"], sp["K"], sp["N"]
+        if args.no_tune:
+            cfg = qg.qgemm_plan(qg.OP_W4A16, M, N, K, gs, hz)
+        else:
+            cfg = qg.qgemm_tune(qg.OP_W4A16, sp["A"], sp["W"][0], sp["S"], sp["Z"], sp["C"],
+                                M, N, K, gs, hz, reps=args.tune_reps)
+        sp["cfg"] = cfg
+        tuned.append({"shape": [M, K, N], **{k: cfg[k] for k in ("path", "rows", "bm", "bn",
+                                                                   "bk", "stages", "split_k")}})
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+
+    def step(i, events=None):
+        for j, sp in enumerate(per_shape):
+            W = sp["W"][i % n_sets]
+            if events is not None:
+                events[j][0].record(stream)
+            qg.qgemm_w4a16(sp["A"], W, sp["S"], sp["Z"], C=sp["C"], group_size=gs)
+            if events is not None:
+                events[j][1].record(stream)
+
+    warmup = max(3, args.warmup)
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in per_shape] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(warmup + i, ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world, dev)
+    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(total_ms, world, dev)
+    shape_ms = [statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps))
+                for j in range(len(per_shape))]
+
+    flops_step = sum(shape_flops(s["M"], s["K"], s["N"]) for s in per_shape)
+    bytes_step = sum(shape_bytes(op, s["M"], s["K"], s["N"], hz) for s in per_shape)
+    ms_per_step = total_ms / args.steps
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- end to end: host A in, host C out, through the same entry point ----
+    e2e = run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step)
+
+    # ---- roofline of the dominant call ----
+    j = int(np.argmax(shape_ms))
+    sp = per_shape[j]
+    M, K, N = sp["M"], sp["K"], sp["N"]
+    fl = shape_flops(M, K, N)
+    by = shape_bytes(op, M, K, N, hz)
+    ms = shape_ms[j]
+    intensity = fl / by
+    timed_alone = total_ms < 1000.0
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)   # flop per byte
+    if intensity >= ridge:
+        peak = peaks["bf16_tflops"] if timed_alone else peaks["bf16_tflops_sustained"]
+        achieved = fl / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+    else:
+        achieved = by / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    roof["traffic"] = args.traffic
+    roof["kernel_shape"] = [M, K, N]
+    roof["peak_source"] = (f"{peaks['source']} "
+                           f"({'burst' if timed_alone else 'sustained'} for tensor peaks)")
+
+    details = []
+    for s, t in zip(per_shape, shape_ms):
+        fl_s = shape_flops(s["M"], s["K"], s["N"])
+        by_s = shape_bytes(op, s["M"], s["K"], s["N"], hz)
+        details.append({"shape_mkn": [s["M"], s["K"], s["N"]], "us": round(t * 1e3, 2),
+                        "gbs": round(by_s / (t * 1e-3) / 1e9, 1),
+                        "tflops": round(fl_s / (t * 1e-3) / 1e12, 2),
+                        "hbm_frac": round(by_s / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
+
+    out = {
+        "metric": "int4-weight GEMM TFLOP/s & effective HBM GB/s, M=1..16384, N=K=16384",
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16xu4->f32acc->f16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "op": op, "shapes_mkn": [list(s) for s in shapes],
+                   "group_size": gs, "has_zero": hz, "parallelism": f"replicas{world}",
+                   "l2": f"{n_sets} rotating weight sets (>= 3x L2 between reuses)",
+                   "tuned": tuned},
+        "hbm_gbs_effective": round(world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9, 1),
+        "per_shape": details,
+        "roofline": roof,
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * len(per_shape),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return out
+
+
+def run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step):
+    import torch
+    import gemv_w4a16_w8a8_b200 as qg
+    steps = max(1, min(args.steps, 5))
+    h2d = sum(sp["A_host"].numel() * 2 for sp in per_shape)
+    d2h = sum(sp["C_host"].numel() * 2 for sp in per_shape)
+
+    def one(i):
+        for sp in per_shape:
+            sp["A"].copy_(sp["A_host"], non_blocking=True)
+            qg.qgemm_w4a16(sp["A"], sp["W"][i % len(sp["W"])], sp["S"], sp["Z"], C=sp["C"],
+                           group_size=gs)
+            sp["C_host"].copy_(sp["C"], non_blocking=True)
+
+    one(0)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        one(i + 1)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(world * flops_step * steps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ---- oracle arm ------------------------------------------------------------------------------------
+
+def oracle_sample_rates(workload: str, budget_s: float, seed: int = 0):
+    """Time the oracle on a slice of every shape: all of A's rows (at most 64), the first
+    n_s weight rows, sized so the whole pass takes about budget_s seconds. Returns per-shape
+    (flops_done, seconds, description)."""
+    import oracle
+    from gemv_w4a16_w8a8_b200 import synth
+    wl = WORKLOADS[workload]
+    hz, gs = wl["has_zero"], 128
+    threads = oracle.max_threads()
+    per = budget_s / len(wl["shapes"])
+    out = []
+    for si, (M, K, N) in enumerate(wl["shapes"]):
+        m_s = min(M, 64)
+        # probe with a tiny slice, then size the real one to the budget
+        n_s = 8
+        for attempt in range(2):
+            d = synth.w4a16_inputs(m_s, n_s, K, gs, bool(hz), seed=seed + si)
+            Wq = oracle.pack_int4(d["codes"])
+            t = time.perf_counter()
+            oracle.w4a16(d["A"], Wq, d["scales"], d["zeros"], K, gs, nthreads=threads)
+            dt = time.perf_counter() - t
+            if attempt == 0:
+                n_s = int(max(8, min(N, n_s * per / max(dt, 1e-6))))
+        out.append((2.0 * m_s * n_s * K, dt, f"{m_s}x{n_s} of ({M},{K},{N})"))
+    return out, threads
+
+
+def cpu_baseline(workload: str, budget_s: float = 15.0):
+    rates, threads = oracle_sample_rates(workload, budget_s)
+    wl = WORKLOADS[workload]
+    # time the oracle would take for the whole step, shape by shape at its sampled rate
+    est_s = sum(shape_flops(M, K, N) / (f / t) for (M, K, N), (f, t, _) in zip(wl["shapes"], rates))
+    total = sum(shape_flops(M, K, N) for M, K, N in wl["shapes"])
+    return {"value": total / est_s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": "; ".join(desc for _, _, desc in rates) +
+                      f" (fp64 oracle, {sum(t for _, t, _ in rates):.1f} s of CPU time; "
+                      f"each shape's rate applied to its full FLOPs)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    total_flops = sum(shape_flops(M, K, N) for M, K, N in wl["shapes"])
+    per_step_budget = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(max(0, args.warmup)):
+        oracle_sample_rates(args.workload, per_step_budget / 4)
+    est = []
+    threads = 1
+    samples = ""
+    for _ in range(args.steps):
+        rates, threads = oracle_sample_rates(args.workload, per_step_budget)
+        est.append(sum(shape_flops(M, K, N) / (f / t)
+                       for (M, K, N), (f, t, _) in zip(wl["shapes"], rates)))
+        samples = "; ".join(d for _, _, d in rates)
+    ms_per_step = 1e3 * statistics.mean(est)
+    value = total_flops / (ms_per_step * 1e-3) / 1e12
+    return {
+        "impl": "reference",
+        "metric": "int4-weight GEMM TFLOP/s & effective HBM GB/s, M=1..16384, N=K=16384",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "op": wl["op"],
+                   "shapes_mkn": [list(s) for s in wl["shapes"]], "group_size": 128,
+                   "has_zero": wl["has_zero"], "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": samples + " per step; each shape's sampled rate applied to "
+                                             "its full FLOPs"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-tune", action="store_true")
+    ap.add_argument("--tune-reps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+    else:
+        out = run_ours(args, world, rank, local)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

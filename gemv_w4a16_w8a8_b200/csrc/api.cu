@@ -1,0 +1,566 @@
+// C-ABI entry points of the qgemm library: argument checks, configuration choice (pinned
+// table, then heuristic), the split-K output zeroing, the kernel launch and the error word.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "common.cuh"
+
+// Device error word: kernels with bounded waits set it instead of trapping.
+__device__ unsigned int g_qgemm_error_word;
+
+namespace qg {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultSms = 148;   // B200
+constexpr int kMaxSplit = 64;
+
+std::mutex g_mu;
+
+struct DeviceInfo {
+    bool probed = false;
+    bool sm100 = false;
+    int sms = kDefaultSms;
+    unsigned int *err_word = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+using Key = std::tuple<int, int, int, int, int, int>;   // op, M, N, K, gs, has_zero
+std::map<Key, qgemm_config_t> g_pinned;
+bool g_cache_loaded = false;
+
+// ------------------------------------------------------------------------------------------
+qg_status probe_device(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return QG_ERR_CUDA;
+        }
+        d.sm100 = major == 10 && minor == 0;
+        d.sms = sms > 0 ? sms : kDefaultSms;
+        if (d.sm100) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_qgemm_error_word) != cudaSuccess) {
+                cudaGetLastError();
+                return QG_ERR_CUDA;
+            }
+            d.err_word = static_cast<unsigned int *>(p);
+        }
+        d.probed = true;
+    }
+    *out = &d;
+    return d.sm100 ? QG_OK : QG_ERR_NOT_SM100;
+}
+
+int sm_count_or_default()
+{
+    int n = 0, dev = 0, sms = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess || n <= 0 || cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return kDefaultSms;
+    }
+    return sms > 0 ? sms : kDefaultSms;
+}
+
+int effective_gs(int op, int K, int group_size)
+{
+    if (op != QG_OP_W4A16) return K;
+    return group_size <= 0 ? K : group_size;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape / flag rules shared by the matmul entry points, the planner and the tuner.
+qg_status check_shape(int op, int M, int N, int K, int group_size, int has_zero, int split_k)
+{
+    if (op < QG_OP_W4A16 || op > QG_OP_DENSE_F16) return QG_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+    if (split_k > kMaxSplit) return QG_ERR_INVALID_ARG;
+    if (has_zero != 0 && has_zero != 1) return QG_ERR_INVALID_ARG;
+    switch (op) {
+    case QG_OP_W4A16: {
+        if (K % 32) return QG_ERR_UNSUPPORTED_SHAPE;
+        if (group_size < -1) return QG_ERR_INVALID_ARG;
+        const int gs = effective_gs(op, K, group_size);
+        if (gs % 32 || K % gs) return QG_ERR_UNSUPPORTED_SHAPE;
+        break;
+    }
+    case QG_OP_W8A8:
+    case QG_OP_W2A8:
+        if (group_size != -1 && group_size != 0) return QG_ERR_INVALID_ARG;
+        if (has_zero) return QG_ERR_INVALID_ARG;
+        if (K % (op == QG_OP_W2A8 ? 64 : 16)) return QG_ERR_UNSUPPORTED_SHAPE;
+        break;
+    case QG_OP_DENSE_F16:
+        if (has_zero) return QG_ERR_INVALID_ARG;
+        if (K % 8) return QG_ERR_UNSUPPORTED_SHAPE;
+        break;
+    }
+    return QG_OK;
+}
+
+Problem make_problem(int op, const void *A, const void *W, const void *scales,
+                     const void *zeros, void *C, int M, int N, int K, int group_size,
+                     int has_zero)
+{
+    Problem p;
+    p.op = op;
+    p.A = A;
+    p.W = W;
+    p.scales = scales;
+    p.zeros = zeros;
+    p.C = C;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.gs = effective_gs(op, K, group_size);
+    p.has_zero = has_zero;
+    return p;
+}
+
+size_t out_bytes(const Problem &p)
+{
+    const size_t elt = (p.op == QG_OP_W4A16 || p.op == QG_OP_DENSE_F16) ? 2 : 4;
+    return (size_t)p.M * p.N * elt;
+}
+
+bool supports(const Problem &p, const qgemm_config_t &c)
+{
+    switch (c.path) {
+    case QG_PATH_GEMV:
+        if (p.op == QG_OP_W4A16) return gemv_w4a16_supports(p, c);
+        if (p.op == QG_OP_W8A8 || p.op == QG_OP_W2A8) return gemv_int_supports(p, c);
+        return false;
+    case QG_PATH_TC:
+        return tc_supports(p, c);
+    default:
+        return false;
+    }
+}
+
+// ---- heuristic -------------------------------------------------------------------------------
+
+int pick_split(long tiles, long work_units, long min_units_per_split, int sms)
+{
+    int split = 1;
+    while (split < kMaxSplit && tiles * split < 4L * sms &&
+           work_units / (2L * split) >= min_units_per_split)
+        split *= 2;
+    return split;
+}
+
+qgemm_config_t heuristic(const Problem &p, int sms)
+{
+    qgemm_config_t c;
+    std::memset(&c, 0, sizeof(c));
+    c.split_k = 1;
+    // tensor-core GEMM once there are enough tokens to fill its tile
+    qgemm_config_t tc;
+    std::memset(&tc, 0, sizeof(tc));
+    tc.path = QG_PATH_TC;
+    tc.split_k = 1;
+    if (p.op == QG_OP_DENSE_F16 || p.M > 16) {
+        if (tc_supports(p, tc)) return tc;
+    }
+    c.path = QG_PATH_GEMV;
+    if (p.op == QG_OP_W4A16) {
+        c.rows = 32;
+        const int kb = (p.gs % 128 == 0) ? 128 : (p.gs % 64 == 0 ? 64 : 32);
+        const long tiles = (long)((p.N + 31) / 32) * ((p.M + 15) / 16);
+        c.split_k = pick_split(tiles, p.K / kb, 12, sms);
+    } else {
+        c.rows = 4;
+        const int kc = p.op == QG_OP_W2A8 ? 64 : 16;
+        const long tiles = (long)((p.N + 15) / 16) * ((p.M + 3) / 4);
+        c.split_k = pick_split(tiles, p.K / kc, 128, sms);
+    }
+    return c;
+}
+
+// ---- pinned configurations ------------------------------------------------------------------------
+
+bool parse_line(const char *line, Key *k, qgemm_config_t *c)
+{
+    int op, M, N, K, gs, hz;
+    int v[8];
+    if (std::sscanf(line, "%d %d %d %d %d %d %d %d %d %d %d %d %d %d", &op, &M, &N, &K, &gs, &hz,
+                    &v[0], &v[1], &v[2], &v[3], &v[4], &v[5], &v[6], &v[7]) != 14)
+        return false;
+    *k = Key(op, M, N, K, gs, hz);
+    c->path = v[0];
+    c->rows = v[1];
+    c->bm = v[2];
+    c->bn = v[3];
+    c->bk = v[4];
+    c->stages = v[5];
+    c->split_k = v[6];
+    c->swap_ab = v[7];
+    return true;
+}
+
+qg_status load_file_locked(const char *path)
+{
+    FILE *f = std::fopen(path, "r");
+    if (!f) return QG_ERR_INVALID_ARG;
+    char line[512];
+    while (std::fgets(line, sizeof line, f)) {
+        if (line[0] == '#') continue;
+        Key k;
+        qgemm_config_t c;
+        if (!parse_line(line, &k, &c)) continue;
+        Problem p = make_problem(std::get<0>(k), nullptr, nullptr, nullptr, nullptr, nullptr,
+                                 std::get<1>(k), std::get<2>(k), std::get<3>(k), std::get<4>(k),
+                                 std::get<5>(k));
+        if (check_shape(std::get<0>(k), std::get<1>(k), std::get<2>(k), std::get<3>(k),
+                        std::get<4>(k), std::get<5>(k), c.split_k) == QG_OK &&
+            c.split_k >= 1 && supports(p, c))
+            g_pinned[k] = c;   // entries that cannot run are skipped
+    }
+    std::fclose(f);
+    return QG_OK;
+}
+
+void ensure_cache_loaded_locked()
+{
+    if (g_cache_loaded) return;
+    g_cache_loaded = true;
+    const char *path = std::getenv("QGEMM_CONFIG_CACHE");
+    if (path && *path) load_file_locked(path);
+}
+
+Key key_of(const Problem &p)
+{
+    return Key(p.op, p.M, p.N, p.K, p.gs, p.has_zero);
+}
+
+qgemm_config_t choose(const Problem &p, int split_k, int sms)
+{
+    qgemm_config_t c;
+    bool found = false;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        ensure_cache_loaded_locked();
+        auto it = g_pinned.find(key_of(p));
+        if (it != g_pinned.end()) {
+            c = it->second;
+            found = true;
+        }
+    }
+    if (!found) c = heuristic(p, sms);
+    if (split_k > 0) c.split_k = split_k;
+    return c;
+}
+
+// ---- dispatch ---------------------------------------------------------------------------------------
+
+qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStream_t stream)
+{
+    if (!supports(p, c)) return QG_ERR_BAD_CONFIG;
+    if (c.split_k > 1) {
+        if (cudaMemsetAsync(p.C, 0, out_bytes(p), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return QG_ERR_CUDA;
+        }
+    }
+    cudaError_t e = cudaErrorInvalidValue;
+    if (c.path == QG_PATH_GEMV) {
+        e = (p.op == QG_OP_W4A16) ? launch_gemv_w4a16(p, c, stream) : launch_gemv_int(p, c, stream);
+    } else if (c.path == QG_PATH_TC) {
+        e = launch_tc(p, c, d->err_word, stream);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+qg_status matmul(int op, const void *A, const void *W, const void *scales, const void *zeros,
+                 void *C, int M, int N, int K, int group_size, int split_k, int has_zero,
+                 cudaStream_t stream)
+{
+    qg_status s = check_shape(op, M, N, K, group_size, has_zero, split_k);
+    if (s != QG_OK) return s;
+    if (!A || !W || !C) return QG_ERR_INVALID_ARG;
+    if (op == QG_OP_W4A16) {
+        if (!scales) return QG_ERR_INVALID_ARG;
+        if ((zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+        if (!aligned(scales, 2) || (zeros && !aligned(zeros, 2))) return QG_ERR_ALIGNMENT;
+    }
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    Problem p = make_problem(op, A, W, scales, zeros, C, M, N, K, group_size, has_zero);
+    return run(p, choose(p, split_k, d->sms), d, stream);
+}
+
+std::vector<qgemm_config_t> candidates(const Problem &p)
+{
+    std::vector<qgemm_config_t> out;
+    qgemm_config_t c;
+    std::memset(&c, 0, sizeof(c));
+    if (p.op == QG_OP_W4A16 || p.op == QG_OP_W8A8 || p.op == QG_OP_W2A8) {
+        c.path = QG_PATH_GEMV;
+        const int rows16[] = {16, 32, 64};
+        const int rows_int[] = {1, 2, 4, 8};
+        const int *rows = p.op == QG_OP_W4A16 ? rows16 : rows_int;
+        const int nrows = p.op == QG_OP_W4A16 ? 3 : 4;
+        for (int r = 0; r < nrows; ++r)
+            for (int s = 1; s <= 16; s *= 2) {
+                c.rows = rows[r];
+                c.split_k = s;
+                if (supports(p, c)) out.push_back(c);
+            }
+    }
+    qgemm_config_t t;
+    std::memset(&t, 0, sizeof(t));
+    t.path = QG_PATH_TC;
+    t.split_k = 1;
+    if (tc_supports(p, t)) out.push_back(t);
+    return out;
+}
+
+} // namespace
+} // namespace qg
+
+using namespace qg;
+
+extern "C" {
+
+qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, const void *zeros,
+                      void *C, int M, int N, int K, int group_size, int split_k, int has_zero,
+                      cudaStream_t stream)
+{
+    return matmul(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, split_k, has_zero,
+                  stream);
+}
+
+qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N, int K,
+                     int group_size, int split_k, int has_zero, cudaStream_t stream)
+{
+    return matmul(QG_OP_W8A8, A, W, nullptr, nullptr, C, M, N, K, group_size, split_k, has_zero,
+                  stream);
+}
+
+qg_status qgemm_w2a8(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int N, int K,
+                     int group_size, int split_k, int has_zero, cudaStream_t stream)
+{
+    return matmul(QG_OP_W2A8, A, Wq, nullptr, nullptr, C, M, N, K, group_size, split_k, has_zero,
+                  stream);
+}
+
+qg_status qgemm_dense_f16(const void *A, const void *W, void *C, int M, int N, int K,
+                          int split_k, cudaStream_t stream)
+{
+    return matmul(QG_OP_DENSE_F16, A, W, nullptr, nullptr, C, M, N, K, -1, split_k, 0, stream);
+}
+
+qg_status quant_pack_int4(const uint8_t *codes, uint32_t *packed, int M, int N, int K,
+                          int group_size, int split_k, int has_zero, cudaStream_t stream)
+{
+    (void)M; (void)group_size; (void)split_k; (void)has_zero;
+    if (!codes || !packed || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+    if (K % 32) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(codes, 16) || !aligned(packed, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_pack_int4(codes, packed, N, K, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+qg_status quant_pack_int2(const int8_t *vals, uint32_t *packed, int M, int N, int K,
+                          int group_size, int split_k, int has_zero, cudaStream_t stream)
+{
+    (void)M; (void)group_size; (void)split_k; (void)has_zero;
+    if (!vals || !packed || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+    if (K % 64) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(vals, 16) || !aligned(packed, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_pack_int2(vals, packed, N, K, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+qg_status qgemm_plan(int op, int M, int N, int K, int group_size, int has_zero, int split_k,
+                     qgemm_config_t *out)
+{
+    if (!out) return QG_ERR_INVALID_ARG;
+    qg_status s = check_shape(op, M, N, K, group_size, has_zero, split_k);
+    if (s != QG_OK) return s;
+    Problem p = make_problem(op, nullptr, nullptr, nullptr, nullptr, nullptr, M, N, K, group_size,
+                             has_zero);
+    *out = choose(p, split_k, sm_count_or_default());
+    return supports(p, *out) ? QG_OK : QG_ERR_BAD_CONFIG;
+}
+
+qg_status qgemm_set_config(int op, int M, int N, int K, int group_size, int has_zero,
+                           const qgemm_config_t *cfg)
+{
+    qg_status s = check_shape(op, M, N, K, group_size, has_zero, cfg ? cfg->split_k : 0);
+    if (s != QG_OK) return s;
+    Problem p = make_problem(op, nullptr, nullptr, nullptr, nullptr, nullptr, M, N, K, group_size,
+                             has_zero);
+    std::lock_guard<std::mutex> lk(g_mu);
+    ensure_cache_loaded_locked();
+    if (!cfg) {
+        g_pinned.erase(key_of(p));
+        return QG_OK;
+    }
+    if (cfg->split_k < 1 || !supports(p, *cfg)) return QG_ERR_BAD_CONFIG;
+    g_pinned[key_of(p)] = *cfg;
+    return QG_OK;
+}
+
+qg_status qgemm_tune(int op, const void *A, const void *W, const void *scales,
+                     const void *zeros, void *C, int M, int N, int K, int group_size,
+                     int has_zero, int reps, cudaStream_t stream, qgemm_config_t *best)
+{
+    qg_status s = check_shape(op, M, N, K, group_size, has_zero, 0);
+    if (s != QG_OK) return s;
+    if (!A || !W || !C || (op == QG_OP_W4A16 && !scales)) return QG_ERR_INVALID_ARG;
+    if (op == QG_OP_W4A16 && (zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (reps <= 0) reps = 20;
+    Problem p = make_problem(op, A, W, scales, zeros, C, M, N, K, group_size, has_zero);
+    std::vector<qgemm_config_t> cands = candidates(p);
+    if (cands.empty()) return QG_ERR_BAD_CONFIG;
+    cudaEvent_t e0, e1;
+    if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    float best_ms = 1e30f;
+    qgemm_config_t winner = cands[0];
+    qg_status result = QG_OK;
+    for (const qgemm_config_t &c : cands) {
+        for (int i = 0; i < 2 && result == QG_OK; ++i) result = run(p, c, d, stream);
+        if (result != QG_OK) break;
+        cudaEventRecord(e0, stream);
+        for (int i = 0; i < reps && result == QG_OK; ++i) result = run(p, c, d, stream);
+        cudaEventRecord(e1, stream);
+        if (result != QG_OK || cudaEventSynchronize(e1) != cudaSuccess) {
+            if (result == QG_OK) result = QG_ERR_CUDA;
+            break;
+        }
+        float ms = 0.f;
+        cudaEventElapsedTime(&ms, e0, e1);
+        if (ms < best_ms) {
+            best_ms = ms;
+            winner = c;
+        }
+    }
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    cudaGetLastError();
+    if (result != QG_OK) return result;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        ensure_cache_loaded_locked();
+        g_pinned[key_of(p)] = winner;
+    }
+    if (best) *best = winner;
+    return QG_OK;
+}
+
+qg_status qgemm_save_configs(const char *path)
+{
+    if (!path) return QG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    FILE *f = std::fopen(path, "w");
+    if (!f) return QG_ERR_INVALID_ARG;
+    std::fprintf(f, "# op M N K group_size has_zero path rows bm bn bk stages split_k swap_ab\n");
+    for (const auto &kv : g_pinned) {
+        const Key &k = kv.first;
+        const qgemm_config_t &c = kv.second;
+        std::fprintf(f, "%d %d %d %d %d %d %d %d %d %d %d %d %d %d\n", std::get<0>(k),
+                     std::get<1>(k), std::get<2>(k), std::get<3>(k), std::get<4>(k),
+                     std::get<5>(k), c.path, c.rows, c.bm, c.bn, c.bk, c.stages, c.split_k,
+                     c.swap_ab);
+    }
+    std::fclose(f);
+    return QG_OK;
+}
+
+qg_status qgemm_load_configs(const char *path)
+{
+    if (!path) return QG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_cache_loaded = true;
+    return load_file_locked(path);
+}
+
+void qgemm_clear_configs(void)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_cache_loaded = true;
+    g_pinned.clear();
+}
+
+qg_status qgemm_sync_check(cudaStream_t stream)
+{
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    unsigned int word = 0;
+    const unsigned int zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_qgemm_error_word, sizeof(word)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_qgemm_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return word ? QG_ERR_DEVICE_TIMEOUT : QG_OK;
+}
+
+const char *qgemm_status_string(qg_status status)
+{
+    switch (status) {
+    case QG_OK: return "ok";
+    case QG_ERR_INVALID_ARG: return "invalid argument";
+    case QG_ERR_ALIGNMENT: return "pointer not aligned as required";
+    case QG_ERR_UNSUPPORTED_SHAPE: return "unsupported K / group_size";
+    case QG_ERR_CUDA: return "CUDA runtime or launch error";
+    case QG_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case QG_ERR_NOT_SM100: return "device is not compute capability 10.0 (B200)";
+    case QG_ERR_BAD_CONFIG: return "configuration cannot run this problem";
+    }
+    return "unknown status";
+}
+
+int qgemm_version(void) { return 100; }
+
+} // extern "C"

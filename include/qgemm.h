@@ -1,0 +1,187 @@
+/*
+ * qgemm: low-bit mixed-precision matrix multiplication for NVIDIA B200 (sm_100a).
+ *
+ *     C[M, N] = A[M, K] . dequant(W[N, K])^T        ("nt": A and W both K-contiguous)
+ *
+ * Operand types follow the BitBLAS Matmul benchmark configuration listing
+ * (microsoft/BitBLAS issue #252, "Default Backend Should be changed into tilelang",
+ * op_configs and the MatmulConfig tuple M, N, K, A_dtype, W_dtype, out_dtype, accum_dtype,
+ * layout "nt", group_size, with_scaling, with_zeros):
+ *   W4A16  fp16 activations x unsigned int4 weights with per-group fp16 scale and optional
+ *          fp16 zero point, fp32 accumulation, fp16 output;
+ *   W8A8   int8 x int8, int32 accumulation and int32 output (an int8 dot product returns
+ *          int32: triton-lang/triton PR #3595, "Convert INT8 MMAV2 accumulator layout",
+ *          review discussion);
+ *   W2A8   int8 activations x two's-complement int2 weights, int32 accumulation and output;
+ *   dense  fp16 x fp16 with fp32 accumulation, fp16 output (the in-library baseline).
+ * Parallel-k (split-K) follows hidet-org/hidet issue #364, "Multi-stage software pipelining
+ * and update parallel k rule": the K reduction is cut into split_k parts whose partial results
+ * are added into C with atomic red.global instructions.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller (for example PyTorch tensors); the
+ *     library never frees or retains them. All operands are row-major and densely packed.
+ *   - Calls are asynchronous and ordered on `stream` (0 = legacy default stream).
+ *   - Arguments are validated before any work is queued; on error nothing is launched and
+ *     no memory is touched. Launch failures return QG_ERR_CUDA. Errors raised by a kernel
+ *     after it started (a bounded wait that ran out) are reported by qgemm_sync_check().
+ *   - split_k > 1 makes the call zero C on `stream` first, then add each part into it
+ *     atomically; fp16 results then depend on the (unspecified) order of the additions,
+ *     int32 results do not. split_k <= 0 selects the tuned or heuristic value for the shape.
+ *   - The library allocates no per-call memory. It allocates once per device at first use a
+ *     4-byte device error word; qgemm_tune() allocates nothing either (it times the caller's
+ *     buffers).
+ *   - Nothing throws across this interface.
+ *   - Every pointer argument named below must be 16-byte aligned, except scales and zeros
+ *     (2-byte aligned).
+ */
+#ifndef QGEMM_H_
+#define QGEMM_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qg_status {
+    QG_OK = 0,
+    QG_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, bad flag value        */
+    QG_ERR_ALIGNMENT = 2,         /* a pointer is not aligned as required                  */
+    QG_ERR_UNSUPPORTED_SHAPE = 3, /* K or group_size violates the divisibility rules       */
+    QG_ERR_CUDA = 4,              /* a CUDA runtime call or a kernel launch failed          */
+    QG_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up a bounded wait (qgemm_sync_check)     */
+    QG_ERR_NOT_SM100 = 6,         /* the current device is not compute capability 10.0     */
+    QG_ERR_BAD_CONFIG = 7         /* a config passed to qgemm_set_config cannot run        */
+} qg_status;
+
+typedef enum qg_op {
+    QG_OP_W4A16 = 0,
+    QG_OP_W8A8 = 1,
+    QG_OP_W2A8 = 2,
+    QG_OP_DENSE_F16 = 3
+} qg_op;
+
+typedef enum qg_path {
+    QG_PATH_AUTO = 0, /* let the library choose                                               */
+    QG_PATH_GEMV = 1, /* small-M streaming kernels (weights read once with 128-bit loads)      */
+    QG_PATH_TC = 2    /* tcgen05 tensor-core GEMM with a TMA multi-stage pipeline (large M)   */
+} qg_path;
+
+/* One launch configuration. Fields a path does not use are ignored (set them to 0). */
+typedef struct qgemm_config_t {
+    int32_t path;    /* qg_path                                                             */
+    int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise)  */
+    int32_t bm;      /* TC: tile extent along M                                              */
+    int32_t bn;      /* TC: tile extent along N                                              */
+    int32_t bk;      /* TC: tile extent along K                                              */
+    int32_t stages;  /* TC: depth of the shared-memory pipeline (2..5)                       */
+    int32_t split_k; /* number of K parts (1 = no atomics)                                   */
+    int32_t swap_ab; /* TC: 1 = weights fill the MMA's M side, tokens its N side             */
+} qgemm_config_t;
+
+/* ---- matmuls ----------------------------------------------------------------------------- */
+
+/*
+ * W4A16. A: fp16 [M, K]. Wq: uint32 [N, K/8], code k of row n at bits 4*(k%8) of word k/8
+ * (unsigned 0..15). scales, zeros: fp16 [N, G], G = K / group_size; zeros must be NULL iff
+ * has_zero == 0 (then z = 0). C: fp16 [M, N].
+ *     C[m, n] = sum_k A[m, k] * (q[n, k] - z[n, k/gs]) * s[n, k/gs]
+ * accumulated in fp32, rounded to fp16 (round-to-nearest-even).
+ * group_size: a multiple of 32 that divides K, or -1 / 0 for one group spanning K.
+ * Requires K % 32 == 0.
+ */
+qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, const void *zeros,
+                      void *C, int M, int N, int K, int group_size, int split_k, int has_zero,
+                      cudaStream_t stream);
+
+/*
+ * W8A8. A: int8 [M, K]. W: int8 [N, K]. C: int32 [M, N] = sum_k A[m,k] * W[n,k], exact
+ * (it wraps modulo 2^32 only if |C| >= 2^31, impossible for K <= 131072).
+ * group_size must be -1 or 0 (no scales) and has_zero 0. Requires K % 16 == 0.
+ */
+qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N, int K,
+                     int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/*
+ * W2A8. A: int8 [M, K]. Wq: uint32 [N, K/16], value k of row n is the two's-complement
+ * 2-bit field at bits 2*(k%16) of word k/16 (values -2..1). C: int32 [M, N], exact.
+ * group_size must be -1 or 0 and has_zero 0. Requires K % 64 == 0.
+ */
+qg_status qgemm_w2a8(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int N, int K,
+                     int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/*
+ * Dense fp16 baseline. A: fp16 [M, K]; W: fp16 [N, K]; C: fp16 [M, N] = A . W^T with fp32
+ * accumulation. Requires K % 8 == 0.
+ */
+qg_status qgemm_dense_f16(const void *A, const void *W, void *C, int M, int N, int K,
+                          int split_k, cudaStream_t stream);
+
+/* ---- weight packing ------------------------------------------------------------------------ */
+
+/*
+ * codes: uint8 [N, K] (only the low 4 bits are used) -> packed: uint32 [N, K/8],
+ *     packed[n, j] = sum_{i<8} (codes[n, 8j+i] & 0xF) << 4i.
+ * M, group_size, split_k and has_zero are accepted for a uniform call shape and ignored.
+ * Requires K % 32 == 0.
+ */
+qg_status quant_pack_int4(const uint8_t *codes, uint32_t *packed, int M, int N, int K,
+                          int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/*
+ * vals: int8 [N, K] holding values -2..1 (only the low 2 bits are used) -> packed: uint32
+ * [N, K/16], packed[n, j] = sum_{i<16} (vals[n, 16j+i] & 3) << 2i. Requires K % 64 == 0.
+ */
+qg_status quant_pack_int2(const int8_t *vals, uint32_t *packed, int M, int N, int K,
+                          int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/* ---- configuration ---------------------------------------------------------------------------- */
+
+/*
+ * Fill *out with the configuration a call with these arguments would launch on the current
+ * device (or on a 148-SM B200 if no device is visible). split_k > 0 overrides the split.
+ * Host-only: launches nothing.
+ */
+qg_status qgemm_plan(int op, int M, int N, int K, int group_size, int has_zero, int split_k,
+                     qgemm_config_t *out);
+
+/* Pin *cfg for this exact problem (NULL removes the entry). Checked before it is stored. */
+qg_status qgemm_set_config(int op, int M, int N, int K, int group_size, int has_zero,
+                           const qgemm_config_t *cfg);
+
+/*
+ * Time every candidate configuration for this problem on the caller's buffers (same meaning
+ * as the matching matmul entry point; C is overwritten, W is read only) and pin the fastest.
+ * `reps` timed launches per candidate (<= 0: 20). The winner is copied to *best if non-NULL.
+ * Synchronises `stream`.
+ */
+qg_status qgemm_tune(int op, const void *A, const void *W, const void *scales,
+                     const void *zeros, void *C, int M, int N, int K, int group_size,
+                     int has_zero, int reps, cudaStream_t stream, qgemm_config_t *best);
+
+/* Pinned configurations as text, one per line; load merges into the table. */
+qg_status qgemm_save_configs(const char *path);
+qg_status qgemm_load_configs(const char *path);
+void qgemm_clear_configs(void);
+
+/* ---- errors ------------------------------------------------------------------------------------ */
+
+/*
+ * Synchronise `stream`, then read and clear the current device's error word. Returns
+ * QG_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the last check,
+ * QG_ERR_CUDA if the synchronisation failed, QG_OK otherwise.
+ */
+qg_status qgemm_sync_check(cudaStream_t stream);
+
+const char *qgemm_status_string(qg_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int qgemm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H_ */

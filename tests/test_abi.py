@@ -1,0 +1,149 @@
+"""The C ABI without a GPU: the library loads, exports exactly what include/qgemm.h declares,
+validates arguments before touching a device, and plans / pins configurations on the host."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gemv_w4a16_w8a8_b200 as qg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_and_binding_agree():
+    names = declared_functions()
+    assert names == set(qg.EXPORTS), names ^ set(qg.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = qg.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert qg.qgemm_version() >= 100
+
+
+def test_status_strings():
+    for code in range(8):
+        assert qg.status_string(code) not in ("", "unknown status")
+    assert qg.status_string(99) == "unknown status"
+
+
+# fake, suitably aligned device addresses: every call below must fail validation (or the
+# device probe) before it could dereference them
+A, W, S, Z, C = (ctypes.c_void_p(0x10000 * i) for i in range(1, 6))
+
+
+def w4(M=1, N=64, K=256, gs=128, split=0, hz=1, a=A, w=W, s=S, z=Z, c=C):
+    return qg.lib().qgemm_w4a16(a, w, s, z if hz else None, c, M, N, K, gs, split, hz, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(M=0), qg.QG_ERR_INVALID_ARG),
+    (dict(N=-1), qg.QG_ERR_INVALID_ARG),
+    (dict(K=0), qg.QG_ERR_INVALID_ARG),
+    (dict(K=100, gs=-1), qg.QG_ERR_UNSUPPORTED_SHAPE),      # K % 32
+    (dict(K=256, gs=48), qg.QG_ERR_UNSUPPORTED_SHAPE),      # gs % 32
+    (dict(K=320, gs=128), qg.QG_ERR_UNSUPPORTED_SHAPE),     # K % gs
+    (dict(gs=-5), qg.QG_ERR_INVALID_ARG),
+    (dict(split=65), qg.QG_ERR_INVALID_ARG),
+    (dict(hz=2), qg.QG_ERR_INVALID_ARG),
+    (dict(a=None), qg.QG_ERR_INVALID_ARG),
+    (dict(s=None), qg.QG_ERR_INVALID_ARG),
+    (dict(a=ctypes.c_void_p(0x10008)), qg.QG_ERR_ALIGNMENT),
+    (dict(c=ctypes.c_void_p(0x10004)), qg.QG_ERR_ALIGNMENT),
+    (dict(s=ctypes.c_void_p(0x10001)), qg.QG_ERR_ALIGNMENT),
+])
+def test_w4a16_validation(kw, status):
+    assert w4(**kw) == status
+
+
+def test_zero_pointer_must_match_flag():
+    L = qg.lib()
+    assert L.qgemm_w4a16(A, W, S, None, C, 1, 64, 256, 128, 0, 1, None) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_w4a16(A, W, S, Z, C, 1, 64, 256, 128, 0, 0, None) == qg.QG_ERR_INVALID_ARG
+
+
+def test_int_paths_validation():
+    L = qg.lib()
+    assert L.qgemm_w8a8(A, W, C, 1, 64, 100, -1, 0, 0, None) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert L.qgemm_w8a8(A, W, C, 1, 64, 128, 128, 0, 0, None) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_w8a8(A, W, C, 1, 64, 128, -1, 0, 1, None) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_w2a8(A, W, C, 1, 64, 96, -1, 0, 0, None) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert L.qgemm_dense_f16(A, W, C, 1, 64, 12, 0, None) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert L.quant_pack_int4(A, W, 0, 4, 48, -1, 1, 0, None) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert L.quant_pack_int2(A, W, 0, 4, 32, -1, 1, 0, None) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert L.quant_pack_int4(None, W, 0, 4, 64, -1, 1, 0, None) == qg.QG_ERR_INVALID_ARG
+
+
+def test_valid_call_without_gpu_fails_loudly():
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+    # arguments are valid, so the call reaches the device probe, which must refuse
+    assert w4() in (qg.QG_ERR_CUDA, qg.QG_ERR_NOT_SM100)
+    assert qg.lib().qgemm_sync_check(None) in (qg.QG_ERR_CUDA, qg.QG_ERR_NOT_SM100)
+
+
+# ---- planning and pinned configurations (host only) ----------------------------------------------
+
+def test_plan_small_m_uses_streaming_kernels():
+    c = qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1)
+    assert c["path"] == qg.PATH_GEMV and c["split_k"] >= 1 and c["rows"] in (16, 32, 64)
+    c = qg.qgemm_plan(qg.OP_W8A8, 1, 16384, 16384)
+    assert c["path"] == qg.PATH_GEMV and c["rows"] in (1, 2, 4, 8)
+    c = qg.qgemm_plan(qg.OP_W2A8, 1, 16384, 16384)
+    assert c["path"] == qg.PATH_GEMV
+
+
+def test_plan_split_override():
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1, split_k=4)["split_k"] == 4
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 100, 1)
+
+
+def test_set_save_load_roundtrip(tmp_path):
+    qg.qgemm_clear_configs()
+    cfg = {"path": qg.PATH_GEMV, "rows": 64, "bm": 0, "bn": 0, "bk": 0, "stages": 0,
+           "split_k": 8, "swap_ab": 0}
+    qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 11008, 128, 0, cfg)
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 11008, 128, 0) == cfg
+    path = str(tmp_path / "cfg.txt")
+    qg.qgemm_save_configs(path)
+    qg.qgemm_clear_configs()
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 11008, 128, 0) != cfg
+    qg.qgemm_load_configs(path)
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 11008, 128, 0) == cfg
+    qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 11008, 128, 0, None)
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 11008, 128, 0) != cfg
+    qg.qgemm_clear_configs()
+
+
+def test_set_config_rejects_configs_that_cannot_run():
+    bad = {"path": qg.PATH_GEMV, "rows": 48, "bm": 0, "bn": 0, "bk": 0, "stages": 0,
+           "split_k": 1, "swap_ab": 0}
+    with pytest.raises(qg.QGemmError) as e:
+        qg.qgemm_set_config(qg.OP_W4A16, 1, 256, 256, 128, 0, bad)
+    assert e.value.status == qg.QG_ERR_BAD_CONFIG
+    bad.update(rows=32, path=7)
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, 1, 256, 256, 128, 0, bad)
+
+
+def test_corrupt_cache_file_is_ignored(tmp_path):
+    p = tmp_path / "bad.txt"
+    p.write_text("# header\nnot a line\n0 1 2\n0 1 256 256 128 0 1 48 0 0 0 0 1 0\n")
+    qg.qgemm_clear_configs()
+    qg.qgemm_load_configs(str(p))     # parses, skips every entry
+    assert qg.qgemm_plan(qg.OP_W4A16, 1, 256, 256, 128, 0)["rows"] != 48
+    qg.qgemm_clear_configs()
