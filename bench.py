@@ -103,6 +103,14 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def wait_first_sample(self, timeout=5.0):
+        t = time.time()
+        while self.proc is not None and time.time() - t < timeout:
+            self.f.flush()
+            if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
+
     def __exit__(self, *exc):
         if self.proc is not None:
             self.proc.terminate()
@@ -120,7 +128,6 @@ class ClockSampler:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) >= 9:
                 rows.append(parts)
-        os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -178,11 +185,8 @@ def run_ours(args, world, rank, local):
     shapes = wl["shapes"]
     peaks = load_peaks()
 
-    # inputs: one A per shape; weights: one packed set per shape, replicated so that a step
-    # never reads weights that an earlier step left in L2
-    step_w_bytes = sum(N * K // 2 for _, K, N in shapes)
-    n_sets = max(1, math.ceil(3 * L2_BYTES / step_w_bytes))
-    n_sets = min(n_sets, 8)
+    # inputs: one A per shape; weights: each shape's packed matrix replicated into enough
+    # copies (>= 3x L2 in total) that consecutive calls of a shape never find theirs in L2
     per_shape = []
     for si, (M, K, N) in enumerate(shapes):
         d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=1000 * si)
@@ -192,9 +196,11 @@ def run_ours(args, world, rank, local):
         Z = torch.from_numpy(d["zeros"]).to(dev) if hz else None
         Wq0 = qg.quant_pack_int4(codes)
         del codes
+        n_sets = max(1, min(64, math.ceil(3 * L2_BYTES / (N * K // 2))))
         sets = [Wq0] + [Wq0.clone() for _ in range(n_sets - 1)]
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         per_shape.append({"M": M, "K": K, "N": N, "A": A, "S": S, "Z": Z, "W": sets, "C": C,
+                          "n_sets": n_sets,
                           "A_host": torch.from_numpy(d["A"]).pin_memory(),
                           "C_host": torch.empty((M, N), dtype=torch.float16).pin_memory()})
         del d
@@ -216,37 +222,75 @@ def run_ours(args, world, rank, local):
 
     stream = torch.cuda.current_stream()
 
-    def step(i, events=None):
-        for j, sp in enumerate(per_shape):
-            W = sp["W"][i % n_sets]
-            if events is not None:
-                events[j][0].record(stream)
-            qg.qgemm_w4a16(sp["A"], W, sp["S"], sp["Z"], C=sp["C"], group_size=gs)
-            if events is not None:
-                events[j][1].record(stream)
+    def call(sp, i):
+        qg.qgemm_w4a16(sp["A"], sp["W"][i % sp["n_sets"]], sp["S"], sp["Z"], C=sp["C"],
+                       group_size=gs)
 
-    warmup = max(3, args.warmup)
-    for i in range(warmup):
-        step(i)
+    n_sets = max(sp["n_sets"] for sp in per_shape)
+
+    # eager warm-up (first calls probe the device), then one CUDA graph per weight set holding
+    # one whole step: the timed loop replays graphs, so host launch overhead stays out of it
+    for i in range(3):
+        for sp in per_shape:
+            call(sp, i)
+    torch.cuda.synchronize()
+    graphs = []
+    for w in range(n_sets):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for sp in per_shape:
+                call(sp, w)
+        graphs.append(g)
+    # per-shape graphs (R back-to-back calls, weight sets cycling) for the per-call timings
+    reps = max(n_sets, 20)
+    reps = min(reps, 64)
+    shape_graphs = []
+    for sp in per_shape:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for r in range(reps):
+                call(sp, r)
+        shape_graphs.append(g)
     torch.cuda.synchronize()
 
-    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-           for _ in per_shape] for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.__enter__()
+    clk.wait_first_sample()
+    warmup = max(3, args.warmup)
+    t_w = time.perf_counter()
+    i = 0
+    while i < warmup or (time.perf_counter() - t_w < 0.5 and i < 100000):
+        graphs[i % n_sets].replay()
+        i += 1
+        if i % 16 == 0:
+            torch.cuda.synchronize()
+    warm_steps = i
+    torch.cuda.synchronize()
+
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier(world, dev)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(warmup + i, ev[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        graphs[(warm_steps + i) % n_sets].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
     barrier(world, dev)
     total_ms = t0.elapsed_time(t1)
     total_ms = max_over_ranks(total_ms, world, dev)
-    shape_ms = [statistics.mean(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps))
-                for j in range(len(per_shape))]
+
+    # per-call device time of every shape, same launch configuration as the step
+    shape_ms = []
+    for g in shape_graphs:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        shape_ms.append(e0.elapsed_time(e1) / reps)
+    clk.__exit__(None, None, None)
 
     flops_step = sum(shape_flops(s["M"], s["K"], s["N"]) for s in per_shape)
     bytes_step = sum(shape_bytes(op, s["M"], s["K"], s["N"], hz) for s in per_shape)
@@ -295,7 +339,7 @@ def run_ours(args, world, rank, local):
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
-        "warmup": warmup,
+        "warmup": warm_steps,
         "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True,
         "scaling": "weak",
@@ -304,13 +348,17 @@ def run_ours(args, world, rank, local):
         "data": "synthetic",
         "config": {"workload": args.workload, "op": op, "shapes_mkn": [list(s) for s in shapes],
                    "group_size": gs, "has_zero": hz, "parallelism": f"replicas{world}",
-                   "l2": f"{n_sets} rotating weight sets (>= 3x L2 between reuses)",
+                   "l2": "rotating weight copies per shape, >= 3x L2 between reuses "
+                         f"({[sp['n_sets'] for sp in per_shape]})",
                    "tuned": tuned},
         "hbm_gbs_effective": round(world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9, 1),
         "per_shape": details,
         "roofline": roof,
         "e2e": e2e,
         "clocks": clk.summary(),
+        "timing": {"step": "CUDA graph of one step replayed back to back (events around the K "
+                           "replays)", "per_shape": f"graph of {reps} back-to-back calls per shape",
+                   "warmup_steps_run": warm_steps},
         "gpu_launches": args.steps * len(per_shape),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -4,6 +4,7 @@
 
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -168,17 +169,43 @@ int pick_split(long tiles, long work_units, long min_units_per_split, int sms)
     return split;
 }
 
+int pow2_at_least(int x, int lo, int hi)
+{
+    int v = lo;
+    while (v < x && v < hi) v *= 2;
+    return v;
+}
+
+int k_per_slab(int op) { return (op == QG_OP_DENSE_F16 || op == QG_OP_W4A16) ? 64 : 128; }
+
+// tensor-core tile for M tokens: the token tile covers M (up to 256); the pipeline is as deep as
+// shared memory allows (at most 4); K is split until the tiles fill every SM once.
+qgemm_config_t tc_default(const Problem &p, int sms)
+{
+    qgemm_config_t c;
+    std::memset(&c, 0, sizeof(c));
+    c.path = QG_PATH_TC;
+    c.bm = 128;
+    c.bn = pow2_at_least(p.M, 16, 256);
+    c.bk = k_per_slab(p.op);
+    c.stages = std::min(4, tc_max_stages(p.op, c.bn));
+    c.swap_ab = 1;
+    const long tiles = (long)((p.N + 127) / 128) * ((p.M + c.bn - 1) / c.bn);
+    const long nkb = (p.K + c.bk - 1) / c.bk;
+    c.split_k = 1;
+    while (c.split_k < 16 && tiles * c.split_k < sms && nkb / (2L * c.split_k) >= 4)
+        c.split_k *= 2;
+    return c;
+}
+
 qgemm_config_t heuristic(const Problem &p, int sms)
 {
     qgemm_config_t c;
     std::memset(&c, 0, sizeof(c));
     c.split_k = 1;
     // tensor-core GEMM once there are enough tokens to fill its tile
-    qgemm_config_t tc;
-    std::memset(&tc, 0, sizeof(tc));
-    tc.path = QG_PATH_TC;
-    tc.split_k = 1;
     if (p.op == QG_OP_DENSE_F16 || p.M > 16) {
+        qgemm_config_t tc = tc_default(p, sms);
         if (tc_supports(p, tc)) return tc;
     }
     c.path = QG_PATH_GEMV;
@@ -332,11 +359,23 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                 if (supports(p, c)) out.push_back(c);
             }
     }
-    qgemm_config_t t;
-    std::memset(&t, 0, sizeof(t));
-    t.path = QG_PATH_TC;
-    t.split_k = 1;
-    if (tc_supports(p, t)) out.push_back(t);
+    if (p.op == QG_OP_DENSE_F16 || p.M > 1) {
+        const qgemm_config_t base = tc_default(p, kDefaultSms);
+        const int bns[2] = {base.bn, base.bn / 2};
+        for (int bi = 0; bi < 2; ++bi) {
+            if (bns[bi] < 16) continue;
+            for (int st = 2; st <= 5; ++st)
+                for (int sk = 1; sk <= 8; sk *= 2) {
+                    qgemm_config_t t = base;
+                    t.bn = bns[bi];
+                    t.stages = st;
+                    t.split_k = sk;
+                    const long tiles = (long)((p.N + 127) / 128) * ((p.M + t.bn - 1) / t.bn);
+                    if (sk > 1 && tiles >= 2L * kDefaultSms) continue;
+                    if (tc_supports(p, t)) out.push_back(t);
+                }
+        }
+    }
     return out;
 }
 

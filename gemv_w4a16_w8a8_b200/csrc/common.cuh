@@ -38,6 +38,8 @@ cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int 
 bool gemv_w4a16_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
 bool tc_supports(const Problem &p, const qgemm_config_t &cfg);
+// Deepest pipeline (2..5) whose shared memory fits for this op and token tile.
+int tc_max_stages(int op, int bn);
 
 // ------------------------------------------------------------------------------------------
 // PTX wrappers

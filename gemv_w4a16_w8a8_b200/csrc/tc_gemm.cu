@@ -1,13 +1,617 @@
-// tcgen05 tensor-core GEMM family (large M). Not built yet: no configuration reaches it.
+// tcgen05 tensor-core GEMM family for the compute-bound regime (M from a few dozen tokens up).
+//
+//   D[128 weight rows, BN tokens] = W_tile[128, K] . A_tile[BN, K]^T     (both K-contiguous)
+//
+// The weights fill the MMA's 128-row M side and the tokens its N side (16..256), so the per-FLOP
+// cost of dequantising weights falls as the token tile grows. One CTA (256 threads) per output
+// tile, warp-specialised:
+//   warp 0      TMA producer: a ring of `STAGES` shared-memory stages, each holding one 128-byte
+//               wide k-slab of the weight tile and of the activation tile (SWIZZLE_128B), tracked
+//               by mbarriers with transaction counts (multi-stage software pipelining, hidet-org/
+//               hidet issue #364; the stage count is a tunable, as the issue's num_stages);
+//   warp 1      allocates the TMEM accumulator, issues tcgen05.mma (kind::f16 for fp16 operands,
+//               kind::i8 for int8 operands) from one thread and commits each stage back to the
+//               producer;
+//   warps 4-7   for packed weights, upcast the packed slab to fp16 / int8 directly into the
+//               canonical K-major SWIZZLE_128B layout the MMA reads (LOP3 magic-number upcast,
+//               PRMT re-ordering); then, for every mode, the epilogue: tcgen05.ld of the fp32 /
+//               int32 accumulator, conversion, and a store or, for split-K, red.global.add.
+// Every wait is bounded (%globaltimer); a wait that runs out raises the device error word, makes
+// the other roles stop, lets in-flight copies land, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 
 namespace qg {
+namespace {
 
-bool tc_supports(const Problem &, const qgemm_config_t &) { return false; }
+enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3 };
 
-cudaError_t launch_tc(const Problem &, const qgemm_config_t &, unsigned int *, cudaStream_t)
+constexpr int kThreads = 256;
+constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
+constexpr int kSlabBytes = 128;        // bytes of K per stage and row (64 fp16 / 128 int8)
+constexpr int kGroupT = 8;             // token tiles per raster group
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
-    return cudaErrorNotSupported;
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete. Gives up after the time
+// limit (raising the error word and the CTA's abort flag) or when another role gave up.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       unsigned int *err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            if (err) atomicOr(err, 1u);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, SWIZZLE_128B, 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);          // start address
+    d |= (uint64_t)1 << 16;                          // leading byte offset (unused here)
+    d |= (uint64_t)(1024 >> 4) << 32;                // stride byte offset: next 8 rows
+    d |= (uint64_t)1 << 46;                          // descriptor version
+    d |= (uint64_t)2 << 61;                          // swizzle: 128B
+    return d;
+}
+
+template <int MODE>
+__device__ __forceinline__ void mma_issue(uint32_t dtm, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    if constexpr (MODE == kDense || MODE == kW4A16) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtm),
+                     "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+                     : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtm),
+                     "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+                     : "memory");
+    }
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                   "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                   "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Instruction descriptor: dense, K-major A and B, M = 128, N = BN.
+//   fp16 x fp16 -> fp32: D format 1, A/B format 0.   int8 x int8 -> int32: D 2, A/B 1 (signed).
+template <int MODE, int BN>
+__host__ __device__ constexpr uint32_t instr_desc()
+{
+    constexpr bool i8 = (MODE == kW8A8 || MODE == kW2A8);
+    return (i8 ? 2u : 1u) << 4 | (i8 ? 1u : 0u) << 7 | (i8 ? 1u : 0u) << 10 |
+           (uint32_t)(BN >> 3) << 17 | (uint32_t)(kRowsW >> 4) << 24;
+}
+
+template <int MODE> struct Traits {
+    static constexpr bool packed = (MODE == kW4A16 || MODE == kW2A8);
+    static constexpr int w_tma_bytes = packed ? kRowsW * 32 : kRowsW * kSlabBytes;
+    static constexpr int w_mma_bytes = packed ? kRowsW * kSlabBytes : 0;   // dequant target
+    static constexpr int k_per_slab = (MODE == kDense || MODE == kW4A16) ? 64 : 128;
+    static constexpr int c_bytes = (MODE == kDense || MODE == kW4A16) ? 2 : 4;
+};
+
+template <int MODE, int BN, int STAGES> struct Smem {
+    static constexpr int w_tma = Traits<MODE>::w_tma_bytes;
+    static constexpr int w_mma = Traits<MODE>::w_mma_bytes;
+    static constexpr int a_bytes = BN * kSlabBytes;
+    static constexpr int stage = w_tma + w_mma + a_bytes;
+    static constexpr int bars = 8 * (3 * STAGES + 1) + 16;
+    static constexpr int total = 1024 + STAGES * stage + bars;
+};
+
+template <int BN> constexpr uint32_t tmem_cols() { return BN < 32 ? 32u : (uint32_t)BN; }
+
+// Upcast one 128-row slab of packed int4 (8 words per row) into fp16 (q - z) * s, written in
+// the SWIZZLE_128B K-major layout. Thread r owns weight row r of the tile.
+__device__ __forceinline__ void dequant_w4(const uint32_t *packed, uint8_t *dst, int r,
+                                           uint32_t sz0, uint32_t sz1, uint32_t nz0, uint32_t nz1)
+{
+    constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
+    constexpr uint32_t kInv16 = 0x2C002C00u, kNeg64 = 0xD400D400u;
+    const uint4 p0 = *reinterpret_cast<const uint4 *>(packed + r * 8);
+    const uint4 p1 = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4);
+    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t w = words[j], w8 = w >> 8;
+        const uint32_t h0 = hsub2_u32(lop3_and_or(w, kLo, kMagic), kMagic);        // q0 q4
+        const uint32_t h1 = hfma2_u32(lop3_and_or(w, kHi, kMagic), kInv16, kNeg64); // q1 q5
+        const uint32_t h2 = hsub2_u32(lop3_and_or(w8, kLo, kMagic), kMagic);       // q2 q6
+        const uint32_t h3 = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);// q3 q7
+        const uint32_t s = j < 4 ? sz0 : sz1, nz = j < 4 ? nz0 : nz1;
+        uint4 o;
+        o.x = hfma2_u32(prmt(h0, h1, 0x5410), s, nz);   // (q0, q1)
+        o.y = hfma2_u32(prmt(h2, h3, 0x5410), s, nz);   // (q2, q3)
+        o.z = hfma2_u32(prmt(h0, h1, 0x7632), s, nz);   // (q4, q5)
+        o.w = hfma2_u32(prmt(h2, h3, 0x7632), s, nz);   // (q6, q7)
+        *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = o;
+    }
+}
+
+// Upcast one slab of packed int2 (8 words = 128 values per row) into int8 values -2..1.
+__device__ __forceinline__ void dequant_w2(const uint32_t *packed, uint8_t *dst, int r)
+{
+    const uint4 p0 = *reinterpret_cast<const uint4 *>(packed + r * 8);
+    const uint4 p1 = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4);
+    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t wf = words[j] ^ 0xAAAAAAAAu;           // u' = u ^ 2, value = u' - 2
+        const uint32_t f0 = wf & 0x03030303u;                 // fields 0, 4, 8, 12
+        const uint32_t f1 = (wf >> 2) & 0x03030303u;          // fields 1, 5, 9, 13
+        const uint32_t f2 = (wf >> 4) & 0x03030303u;
+        const uint32_t f3 = (wf >> 6) & 0x03030303u;
+        // 4x4 byte transpose -> natural order (fields 4i .. 4i+3 in register i)
+        const uint32_t t0 = prmt(f0, f1, 0x5140), t1 = prmt(f0, f1, 0x7362);
+        const uint32_t t2 = prmt(f2, f3, 0x5140), t3 = prmt(f2, f3, 0x7362);
+        uint4 o;
+        o.x = prmt(t0, t2, 0x5410);
+        o.y = prmt(t0, t2, 0x7632);
+        o.z = prmt(t1, t3, 0x5410);
+        o.w = prmt(t1, t3, 0x7632);
+        // per byte: (u' + 0x7E) ^ 0x80 = u' - 2 (no carry leaves a byte: u' + 0x7E <= 0x81)
+        o.x = (o.x + 0x7E7E7E7Eu) ^ 0x80808080u;
+        o.y = (o.y + 0x7E7E7E7Eu) ^ 0x80808080u;
+        o.z = (o.z + 0x7E7E7E7Eu) ^ 0x80808080u;
+        o.w = (o.w + 0x7E7E7E7Eu) ^ 0x80808080u;
+        *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = o;
+    }
+}
+
+__device__ __forceinline__ uint32_t half2_bcast(float x)
+{
+    const uint16_t b = half_bits_rn(x);
+    return (uint32_t)b | ((uint32_t)b << 16);
+}
+
+template <int MODE, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
+               const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
+               int M, int N, int K, int gs, int kb_per_split, int atomic_out, unsigned int *err)
+{
+    using T = Traits<MODE>;
+    using L = Smem<MODE, BN, STAGES>;
+    constexpr uint32_t kCols = tmem_cols<BN>();
+    constexpr uint32_t kIdesc = instr_desc<MODE, BN>();
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * L::stage);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // tile coordinates: token-tile groups of kGroupT, weight tiles fastest inside a group
+    const int n_tiles = (N + kRowsW - 1) / kRowsW;
+    const int t_tiles = (M + BN - 1) / BN;
+    const int bid = blockIdx.x;
+    const int per_group = kGroupT * n_tiles;
+    const int group = bid / per_group;
+    const int first_t = group * kGroupT;
+    const int gt = min(kGroupT, t_tiles - first_t);
+    const int within = bid - group * per_group;
+    const int t_tile = first_t + within % gt;
+    const int n_tile = within / gt;
+    const int n0 = n_tile * kRowsW;
+    const int t0 = t_tile * BN;
+
+    const int nkb = (K + T::k_per_slab - 1) / T::k_per_slab;
+    const int kb0 = blockIdx.y * kb_per_split;
+    const int kb1 = min(nkb, kb0 + kb_per_split);
+    if (kb0 >= kb1) return;          // empty split (C was zeroed by the host)
+    const int nk = kb1 - kb0;
+
+    auto full_bar = [&](int s) { return smem_u32(bars + s); };
+    auto deq_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+    auto empty_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
+    const uint32_t accum_bar = smem_u32(bars + 3 * STAGES);
+    auto w_tma = [&](int s) { return base + s * L::stage; };
+    auto w_mma = [&](int s) { return base + s * L::stage + L::w_tma; };
+    auto a_tile = [&](int s) { return base + s * L::stage + L::w_tma + L::w_mma; };
+
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(deq_bar(s), 128);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(accum_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_proxy_async_smem();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_holder)),
+                     "r"(kCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            constexpr uint32_t kTx = L::w_tma + L::a_bytes;
+            const int wx_per_kb = Traits<MODE>::packed ? 8 : T::k_per_slab;   // x units of tm_w
+            int issued = 0;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                const uint32_t ph = (i / STAGES) & 1;
+                if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, err)) break;
+                mbar_expect_tx(full_bar(s), kTx);
+                const int kb = kb0 + i;
+                tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * wx_per_kb, n0);
+                tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kb * T::k_per_slab, t0);
+                ++issued;
+            }
+            // let every copy this thread started land before the CTA can exit
+            for (int i = max(0, issued - STAGES); i < issued; ++i) {
+                int dummy_abort = 0;
+                mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                const uint32_t ph = (i / STAGES) & 1;
+                if (!mbar_wait(full_bar(s), ph, abort_flag, err)) break;
+                if constexpr (T::packed) {
+                    if (!mbar_wait(deq_bar(s), ph, abort_flag, err)) break;
+                }
+                tc_fence_after();
+                const uint32_t a_base = smem_u32(T::packed ? w_mma(s) : w_tma(s));
+                const uint64_t adesc = sw128_desc(a_base);
+                const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
+                    mma_issue<MODE>(tmem_d, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                    (i | k) != 0 ? 1u : 0u);
+                mma_commit(empty_bar(s));
+            }
+            mma_commit(accum_bar);
+        }
+    } else if (warp >= 4) {
+        const int r = tid - 128;           // weight row of the tile / TMEM lane
+        // ---------------- dequantisation (packed weights) ----------------
+        if constexpr (T::packed) {
+            const int n = min(n0 + r, N - 1);
+            const int G = K / gs;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % STAGES;
+                const uint32_t ph = (i / STAGES) & 1;
+                if (!mbar_wait(full_bar(s), ph, abort_flag, err)) break;
+                const uint32_t *packed = reinterpret_cast<const uint32_t *>(w_tma(s));
+                if constexpr (MODE == kW4A16) {
+                    const int k0 = (kb0 + i) * 64;
+                    const int g0 = min(k0 / gs, G - 1), g1 = min((k0 + 32) / gs, G - 1);
+                    const float s0 = __half2float(S[(size_t)n * G + g0]);
+                    const float s1 = __half2float(S[(size_t)n * G + g1]);
+                    const float z0 = Z ? __half2float(Z[(size_t)n * G + g0]) : 0.f;
+                    const float z1 = Z ? __half2float(Z[(size_t)n * G + g1]) : 0.f;
+                    dequant_w4(packed, w_mma(s), r, half2_bcast(s0), half2_bcast(s1),
+                               half2_bcast(-z0 * s0), half2_bcast(-z1 * s1));
+                } else {
+                    dequant_w2(packed, w_mma(s), r);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(deq_bar(s));
+            }
+        }
+        // ---------------- epilogue ----------------
+        bool ok = mbar_wait(accum_bar, 0, abort_flag, err);
+        tc_fence_after();
+        // tcgen05.ld is warp-collective: decide per warp, never per lane
+        ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+        if (ok) {
+            const int n = n0 + r;
+            const uint32_t lane_addr = tmem_d + ((uint32_t)((warp - 4) * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                uint32_t v[16];
+                tmem_ld16(lane_addr + c, v);
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = t0 + c + j;
+                        if (t < M) {
+                            if constexpr (T::c_bytes == 2) {
+                                __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
+                                const float x = __uint_as_float(v[j]);
+                                if (atomic_out) red_add_f16(dst, half_bits_rn(x));
+                                else *dst = __float2half_rn(x);
+                            } else {
+                                int32_t *dst = static_cast<int32_t *>(C) + (size_t)t * N + n;
+                                if (atomic_out) red_add_s32(dst, (int)v[j]);
+                                else *dst = (int)v[j];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
+                     "r"(kCols)
+                     : "memory");
+    }
+}
+
+// ---- host side -----------------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
+              uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle sw)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int mode_of(int op)
+{
+    switch (op) {
+    case QG_OP_DENSE_F16: return kDense;
+    case QG_OP_W8A8: return kW8A8;
+    case QG_OP_W4A16: return kW4A16;
+    default: return kW2A8;
+    }
+}
+
+int smem_bytes(int mode, int bn, int stages)
+{
+    const bool packed = (mode == kW4A16 || mode == kW2A8);
+    const int stage = (packed ? kRowsW * 32 + kRowsW * kSlabBytes : kRowsW * kSlabBytes) +
+                      bn * kSlabBytes;
+    return 1024 + stages * stage + 8 * (3 * stages + 1) + 16;
+}
+
+constexpr int kMaxSmem = 227 * 1024;
+
+template <int MODE, int BN, int STAGES>
+cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
+{
+    using T = Traits<MODE>;
+    using L = Smem<MODE, BN, STAGES>;
+    if (L::total > kMaxSmem) return cudaErrorInvalidConfiguration;
+    auto kern = tc_gemm_kernel<MODE, BN, STAGES>;
+    // the dynamic shared-memory opt-in is per device: remember it per device
+    static std::mutex mu;
+    static bool opted_in[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!opted_in[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 L::total);
+            if (e != cudaSuccess) return e;
+            opted_in[dev] = true;
+        }
+    }
+
+    CUtensorMap tw, ta;
+    bool ok;
+    if constexpr (MODE == kDense) {
+        ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.W, p.K, p.N, (uint64_t)p.K * 2, 64,
+                      kRowsW, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
+                      BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else if constexpr (MODE == kW8A8) {
+        ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.W, p.K, p.N, (uint64_t)p.K, 128,
+                      kRowsW, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    } else if constexpr (MODE == kW4A16) {
+        ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
+                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
+                      BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 16, p.N, (uint64_t)p.K / 4,
+                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+
+    const int nkb = (p.K + T::k_per_slab - 1) / T::k_per_slab;
+    const int kbps = (nkb + split_k - 1) / split_k;
+    const int splits = (nkb + kbps - 1) / kbps;
+    const int n_tiles = (p.N + kRowsW - 1) / kRowsW;
+    const int t_tiles = (p.M + BN - 1) / BN;
+    dim3 grid(n_tiles * t_tiles, splits);
+    kern<<<grid, kThreads, L::total, stream>>>(
+        tw, ta, static_cast<const __half *>(p.scales),
+        p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, p.C, p.M, p.N, p.K, p.gs,
+        kbps, split_k > 1 ? 1 : 0, err);
+    return cudaGetLastError();
+}
+
+template <int MODE, int BN>
+cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                          cudaStream_t stream)
+{
+    switch (c.stages) {
+    case 2: return launch_t<MODE, BN, 2>(p, c.split_k, err, stream);
+    case 3: return launch_t<MODE, BN, 3>(p, c.split_k, err, stream);
+    case 4: return launch_t<MODE, BN, 4>(p, c.split_k, err, stream);
+    case 5: return launch_t<MODE, BN, 5>(p, c.split_k, err, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int MODE>
+cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                      cudaStream_t stream)
+{
+    switch (c.bn) {
+    case 16: return launch_stages<MODE, 16>(p, c, err, stream);
+    case 32: return launch_stages<MODE, 32>(p, c, err, stream);
+    case 64: return launch_stages<MODE, 64>(p, c, err, stream);
+    case 128: return launch_stages<MODE, 128>(p, c, err, stream);
+    case 256: return launch_stages<MODE, 256>(p, c, err, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+} // namespace
+
+bool tc_supports(const Problem &p, const qgemm_config_t &c)
+{
+    if (c.path != QG_PATH_TC) return false;
+    if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
+    if (c.stages < 2 || c.stages > 5) return false;
+    if (c.split_k < 1 || c.split_k > 64) return false;
+    if (smem_bytes(mode_of(p.op), c.bn, c.stages) > kMaxSmem) return false;
+    if (p.op == QG_OP_W4A16 && (p.K % 32 || p.gs % 32 || p.K % p.gs)) return false;
+    if (p.op == QG_OP_W2A8 && p.K % 64) return false;
+    if (p.op == QG_OP_W8A8 && p.K % 16) return false;
+    if (p.op == QG_OP_DENSE_F16 && p.K % 8) return false;
+    return true;
+}
+
+int tc_max_stages(int op, int bn)
+{
+    int s = 5;
+    while (s > 2 && smem_bytes(mode_of(op), bn, s) > kMaxSmem) --s;
+    return s;
+}
+
+cudaError_t launch_tc(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                      cudaStream_t stream)
+{
+    switch (mode_of(p.op)) {
+    case kDense: return launch_bn<kDense>(p, c, err, stream);
+    case kW8A8: return launch_bn<kW8A8>(p, c, err, stream);
+    case kW4A16: return launch_bn<kW4A16>(p, c, err, stream);
+    default: return launch_bn<kW2A8>(p, c, err, stream);
+    }
 }
 
 } // namespace qg

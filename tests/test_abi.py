@@ -147,3 +147,39 @@ def test_corrupt_cache_file_is_ignored(tmp_path):
     qg.qgemm_load_configs(str(p))     # parses, skips every entry
     assert qg.qgemm_plan(qg.OP_W4A16, 1, 256, 256, 128, 0)["rows"] != 48
     qg.qgemm_clear_configs()
+
+
+# ---- tensor-core path planning (host only) ---------------------------------------------------------
+
+def _tc(bn, stages, split=1):
+    return {"path": qg.PATH_TC, "rows": 0, "bm": 128, "bn": bn, "bk": 0, "stages": stages,
+            "split_k": split, "swap_ab": 1}
+
+
+def test_plan_large_m_uses_tensor_cores():
+    c = qg.qgemm_plan(qg.OP_W4A16, 16384, 16384, 16384, 128, 1)
+    assert c["path"] == qg.PATH_TC and c["bn"] == 256 and 2 <= c["stages"] <= 5
+    assert c["split_k"] == 1                     # 8192 tiles fill the GPU many times
+    c = qg.qgemm_plan(qg.OP_W4A16, 32, 16384, 16384, 128, 1)
+    assert c["path"] == qg.PATH_TC and c["bn"] == 32 and c["split_k"] >= 1
+    c = qg.qgemm_plan(qg.OP_DENSE_F16, 1, 256, 256)
+    assert c["path"] == qg.PATH_TC and c["bn"] == 16
+    for op in (qg.OP_W8A8, qg.OP_W2A8):
+        assert qg.qgemm_plan(op, 512, 16384, 16384)["path"] == qg.PATH_TC
+
+
+def test_tc_split_fills_the_gpu():
+    c = qg.qgemm_plan(qg.OP_W4A16, 128, 4096, 4096, 128, 1)   # 32 tiles -> split
+    assert c["path"] == qg.PATH_TC and c["split_k"] >= 4
+
+
+def test_tc_config_limits():
+    M, N, K = 256, 512, 1024
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 4))      # 214 KB of smem
+    for bad in (_tc(256, 5), _tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, bad)
+    qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 4))
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 5))
+    qg.qgemm_clear_configs()
