@@ -157,6 +157,14 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def job_throughput(local_ms: float, flops_per_step: float, steps: int, world: int,
+                   device=None) -> tuple[float, float]:
+    """Whole-job TFLOP/s: every rank ran `steps` steps of `flops_per_step`; the job took as
+    long as its slowest rank. Returns (value, max_ms)."""
+    max_ms = max_over_ranks(local_ms, world, device)
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12, max_ms
+
+
 def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
@@ -277,8 +285,7 @@ def run_ours(args, world, rank, local):
     t1.record(stream)
     torch.cuda.synchronize()
     barrier(world, dev)
-    total_ms = t0.elapsed_time(t1)
-    total_ms = max_over_ranks(total_ms, world, dev)
+    local_ms = t0.elapsed_time(t1)
 
     # per-call device time of every shape, same launch configuration as the step
     shape_ms = []
@@ -294,8 +301,8 @@ def run_ours(args, world, rank, local):
 
     flops_step = sum(shape_flops(s["M"], s["K"], s["N"]) for s in per_shape)
     bytes_step = sum(shape_bytes(op, s["M"], s["K"], s["N"], hz) for s in per_shape)
+    value, total_ms = job_throughput(local_ms, flops_step, args.steps, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
 
     # ---- end to end: host A in, host C out, through the same entry point ----
     e2e = run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step)
@@ -394,8 +401,8 @@ def run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step):
         one(i + 1)
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    return {"value": round(world * flops_step * steps / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    value, ms = job_throughput(e0.elapsed_time(e1), flops_step, steps, world, dev)
+    return {"value": round(value, 3), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 

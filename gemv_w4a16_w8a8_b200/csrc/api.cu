@@ -148,7 +148,8 @@ bool supports(const Problem &p, const qgemm_config_t &c)
 {
     switch (c.path) {
     case QG_PATH_GEMV:
-        if (p.op == QG_OP_W4A16) return gemv_w4a16_supports(p, c);
+        if (p.op == QG_OP_W4A16)
+            return c.stages ? gemv_w4a16_tma_supports(p, c) : gemv_w4a16_supports(p, c);
         if (p.op == QG_OP_W8A8 || p.op == QG_OP_W2A8) return gemv_int_supports(p, c);
         return false;
     case QG_PATH_TC:
@@ -214,6 +215,7 @@ qgemm_config_t heuristic(const Problem &p, int sms)
         const int kb = (p.gs % 128 == 0) ? 128 : (p.gs % 64 == 0 ? 64 : 32);
         const long tiles = (long)((p.N + 31) / 32) * ((p.M + 15) / 16);
         c.split_k = pick_split(tiles, p.K / kb, 12, sms);
+        if (p.gs % 128 == 0) c.stages = 4;       // TMA-fed kernel
     } else {
         c.rows = 4;
         const int kc = p.op == QG_OP_W2A8 ? 64 : 16;
@@ -310,7 +312,11 @@ qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStre
     }
     cudaError_t e = cudaErrorInvalidValue;
     if (c.path == QG_PATH_GEMV) {
-        e = (p.op == QG_OP_W4A16) ? launch_gemv_w4a16(p, c, stream) : launch_gemv_int(p, c, stream);
+        if (p.op == QG_OP_W4A16)
+            e = c.stages ? launch_gemv_w4a16_tma(p, c, d->err_word, stream)
+                         : launch_gemv_w4a16(p, c, stream);
+        else
+            e = launch_gemv_int(p, c, stream);
     } else if (c.path == QG_PATH_TC) {
         e = launch_tc(p, c, d->err_word, stream);
     }
@@ -352,12 +358,15 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
         const int rows_int[] = {1, 2, 4, 8};
         const int *rows = p.op == QG_OP_W4A16 ? rows16 : rows_int;
         const int nrows = p.op == QG_OP_W4A16 ? 3 : 4;
+        const int stage_opts[5] = {0, 2, 3, 4, 6};     // 0: register-prefetch kernel
         for (int r = 0; r < nrows; ++r)
-            for (int s = 1; s <= 16; s *= 2) {
-                c.rows = rows[r];
-                c.split_k = s;
-                if (supports(p, c)) out.push_back(c);
-            }
+            for (int st = 0; st < (p.op == QG_OP_W4A16 ? 5 : 1); ++st)
+                for (int s = 1; s <= 16; s *= 2) {
+                    c.rows = rows[r];
+                    c.stages = stage_opts[st];
+                    c.split_k = s;
+                    if (supports(p, c)) out.push_back(c);
+                }
     }
     if (p.op == QG_OP_DENSE_F16 || p.M > 1) {
         const qgemm_config_t base = tc_default(p, kDefaultSms);

@@ -24,6 +24,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace qg {
 namespace {
@@ -34,82 +35,6 @@ constexpr int kThreads = 256;
 constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
 constexpr int kSlabBytes = 128;        // bytes of K per stage and row (64 fp16 / 128 int8)
 constexpr int kGroupT = 8;             // token tiles per raster group
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok)
-                 : "r"(bar), "r"(parity)
-                 : "memory");
-    return ok != 0;
-}
-
-// Wait for the phase of `bar` with the given parity to complete. Gives up after the time
-// limit (raising the error word and the CTA's abort flag) or when another role gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned int *err)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            if (err) atomicOr(err, 1u);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int x, int y)
-{
-    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major, SWIZZLE_128B, 8-row core groups 1024 B apart.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
@@ -403,26 +328,35 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         if (ok) {
             const int n = n0 + r;
             const uint32_t lane_addr = tmem_d + ((uint32_t)((warp - 4) * 32) << 16);
+            // fp16 results leave as (n, n+1) pairs: rows n and n+1 sit in neighbouring lanes
+            const bool pairs = (N & 1) == 0;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
+                if (t0 + c >= M) break;
                 uint32_t v[16];
                 tmem_ld16(lane_addr + c, v);
-                if (n < N) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = t0 + c + j;
-                        if (t < M) {
-                            if constexpr (T::c_bytes == 2) {
-                                __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
-                                const float x = __uint_as_float(v[j]);
-                                if (atomic_out) red_add_f16(dst, half_bits_rn(x));
-                                else *dst = __float2half_rn(x);
-                            } else {
-                                int32_t *dst = static_cast<int32_t *>(C) + (size_t)t * N + n;
-                                if (atomic_out) red_add_s32(dst, (int)v[j]);
-                                else *dst = (int)v[j];
+                for (int j = 0; j < 16; ++j) {
+                    const int t = t0 + c + j;         // the same in every lane
+                    if (t >= M) break;
+                    if constexpr (T::c_bytes == 2) {
+                        const float x = __uint_as_float(v[j]);
+                        const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+                        __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
+                        if (pairs) {
+                            if ((lane & 1) == 0 && n < N) {
+                                const uint32_t h2 = pack_half2_rn(x, y);
+                                if (atomic_out) red_add_f16x2(dst, h2);
+                                else *reinterpret_cast<uint32_t *>(dst) = h2;
                             }
+                        } else if (n < N) {
+                            if (atomic_out) red_add_f16(dst, half_bits_rn(x));
+                            else *dst = __float2half_rn(x);
                         }
+                    } else if (n < N) {
+                        int32_t *dst = static_cast<int32_t *>(C) + (size_t)t * N + n;
+                        if (atomic_out) red_add_s32(dst, (int)v[j]);
+                        else *dst = (int)v[j];
                     }
                 }
             }
@@ -440,38 +374,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 }
 
 // ---- host side -----------------------------------------------------------------------------------
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner,
-              uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
-              CUtensorMapSwizzle sw)
-{
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 int mode_of(int op)
 {

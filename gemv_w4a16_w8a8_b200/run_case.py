@@ -32,7 +32,7 @@ def main(argv=None) -> int:
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--rows", type=int, default=0)
     ap.add_argument("--bn", type=int, default=0)
-    ap.add_argument("--stages", type=int, default=0)
+    ap.add_argument("--stages", type=int, default=-1)
     ap.add_argument("--copies", type=int, default=0, help="weight copies (0: >= 3x L2)")
     a = ap.parse_args(argv)
 
@@ -74,12 +74,13 @@ def main(argv=None) -> int:
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + 2 * M * K + 2 * M * N
 
-    if a.path or a.rows or a.bn or a.stages:
+    if a.path or a.rows or a.bn or a.stages >= 0:
         cfg = qg.qgemm_plan(opc, M, N, K, gs, hz)
-        for key, val in (("path", a.path), ("rows", a.rows), ("bn", a.bn), ("stages", a.stages),
-                         ("split_k", a.split_k)):
+        for key, val in (("path", a.path), ("rows", a.rows), ("bn", a.bn), ("split_k", a.split_k)):
             if val:
                 cfg[key] = val
+        if a.stages >= 0:
+            cfg["stages"] = a.stages
         qg.qgemm_set_config(opc, M, N, K, gs, hz, cfg)
     print("config", qg.qgemm_plan(opc, M, N, K, gs, hz, a.split_k))
 
@@ -102,8 +103,10 @@ def main(argv=None) -> int:
     qg.qgemm_sync_check()
     us = e0.elapsed_time(e1) * 1e3 / a.iters
     flops = 2.0 * M * N * K
+    cfg_used = qg.qgemm_plan(opc, M, N, K, gs, hz, a.split_k)
     print(f"{a.op} M={M} N={N} K={K}: {us:.2f} us/call  {nbytes / us / 1e3:.1f} GB/s  "
-          f"{flops / us / 1e6:.2f} TFLOP/s  ({copies} weight copies)")
+          f"{flops / us / 1e6:.2f} TFLOP/s  ({copies} weight copies)  cfg={cfg_used}")
+    qg.qgemm_set_config(opc, M, N, K, gs, hz, None)
     return 0
 
 

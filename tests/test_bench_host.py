@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py without a GPU: whole-job aggregation over gloo ranks (max over
+ranks, world-size scaling), workload byte / FLOP accounting, and the reference (oracle) arm."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = 10.0 + 5.0 * rank               # rank 1 is the slowest
+        value, max_ms = bench.job_throughput(local_ms, 1e12, 4, world)
+        bench.barrier(world)
+        out[rank] = (value, max_ms)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_job_throughput_is_max_over_ranks(world):
+    mgr = mp.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
+    for rank in range(world):
+        value, max_ms = out[rank]
+        assert max_ms == 15.0
+        # two ranks x 4 steps x 1 TFLOP over the slowest rank's 15 ms
+        assert abs(value - world * 4 * 1e12 / 15e-3 / 1e12) < 1e-9
+
+
+def test_single_rank_needs_no_process_group():
+    value, max_ms = bench.job_throughput(20.0, 2e12, 10, 1)
+    assert max_ms == 20.0 and abs(value - 1000.0) < 1e-9
+
+
+def test_algorithmic_bytes_and_flops():
+    # config 0: M=1, K=N=4096, gs 128, zeros: 8 MiB weights + scales + zeros + A + C
+    b = bench.shape_bytes("w4a16", 1, 4096, 4096, 1)
+    assert b == 4096 * 4096 // 2 + 4096 * 32 * 2 * 2 + 2 * 4096 + 2 * 4096
+    assert bench.shape_bytes("w8a8", 1, 16384, 16384, 0) == 16384 * 16384 + 16384 + 4 * 16384
+    assert bench.shape_bytes("w2a8", 1, 16384, 16384, 0) == 16384 * 16384 // 4 + 16384 + 4 * 16384
+    assert bench.shape_flops(16384, 16384, 16384) == 2.0 * 16384 ** 3
+
+
+def test_reference_arm_prints_one_json_line():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--workload", "w4a16_llama"],
+                       capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0

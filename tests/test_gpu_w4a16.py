@@ -62,9 +62,10 @@ def test_w4a16_split_k_values(split_k):
 
 @pytest.mark.parametrize("rows", [16, 32, 64])
 @pytest.mark.parametrize("M", [1, 12])
-def test_w4a16_each_row_tile(rows, M):
+@pytest.mark.parametrize("stages", [0, 2, 3, 4, 6])
+def test_w4a16_each_row_tile(rows, M, stages):
     case = W4Case(M, 200, 1024, 128, 1, seed=rows)
-    cfg = {"path": qg.PATH_GEMV, "rows": rows, "bm": 0, "bn": 0, "bk": 0, "stages": 0,
+    cfg = {"path": qg.PATH_GEMV, "rows": rows, "bm": 0, "bn": 0, "bk": 0, "stages": stages,
            "split_k": 2, "swap_ab": 0}
     qg.qgemm_set_config(qg.OP_W4A16, M, 200, 1024, 128, 1, cfg)
     try:
@@ -83,8 +84,15 @@ def test_w4a16_one_hot_element_order():
     z = synth.uniform_int((N, G), 0, 15, 7, synth.TID_ZERO, np.int8).astype(np.float16)
     A = np.eye(K, dtype=np.float16)
     for hz in (0, 1):
-        C = qg.qgemm_w4a16(to_dev(A), qg.quant_pack_int4(to_dev(codes)), to_dev(s),
-                           to_dev(z) if hz else None, group_size=gs, split_k=1)
+        # the streaming kernel applies s and z in fp32 per k-block, so the result is exact
+        cfg = {"path": qg.PATH_GEMV, "rows": 32, "bm": 0, "bn": 0, "bk": 0, "stages": 0,
+               "split_k": 1, "swap_ab": 0}
+        qg.qgemm_set_config(qg.OP_W4A16, K, N, K, gs, hz, cfg)
+        try:
+            C = qg.qgemm_w4a16(to_dev(A), qg.quant_pack_int4(to_dev(codes)), to_dev(s),
+                               to_dev(z) if hz else None, group_size=gs, split_k=1)
+        finally:
+            qg.qgemm_set_config(qg.OP_W4A16, K, N, K, gs, hz, None)
         g = np.arange(K) // gs
         want = ((codes.T.astype(np.float64) - (z.T[g].astype(np.float64) if hz else 0.0))
                 * s.T[g].astype(np.float64)).astype(np.float16)
@@ -169,3 +177,18 @@ def test_w4a16_tune_pins_a_working_config():
     finally:
         qg.qgemm_set_config(qg.OP_W4A16, 1, 2048, 4096, 128, 1, None)
     qg.qgemm_sync_check()
+
+
+@pytest.mark.parametrize("stages", [2, 6])
+@pytest.mark.parametrize("split_k", [1, 3, 8])
+def test_w4a16_tma_kernel_long_k(stages, split_k):
+    """K = 16384 through the TMA-fed kernel: many ring wrap-arounds per warp."""
+    M, N, K = 5, 192, 16384
+    case = W4Case(M, N, K, 128, 1, seed=stages + split_k)
+    cfg = {"path": qg.PATH_GEMV, "rows": 64, "bm": 0, "bn": 0, "bk": 0, "stages": stages,
+           "split_k": split_k, "swap_ab": 0}
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, cfg)
+    try:
+        assert_fp16_close(case.run(), case.ref_full(), f"stages={stages} split={split_k}")
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, None)
