@@ -150,6 +150,7 @@ bool supports(const Problem &p, const qgemm_config_t &c)
     case QG_PATH_GEMV:
         if (p.op == QG_OP_W4A16)
             return c.stages ? gemv_w4a16_tma_supports(p, c) : gemv_w4a16_supports(p, c);
+        if (p.op == QG_OP_W2A8 && c.stages) return gemv_w2a8_tma_supports(p, c);
         if (p.op == QG_OP_W8A8 || p.op == QG_OP_W2A8) return gemv_int_supports(p, c);
         return false;
     case QG_PATH_TC:
@@ -189,7 +190,7 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     c.bm = 128;
     c.bn = pow2_at_least(p.M, 16, 256);
     c.bk = k_per_slab(p.op);
-    c.stages = std::min(4, tc_max_stages(p.op, c.bn));
+    c.stages = tc_max_stages(p.op, c.bn);
     c.swap_ab = 1;
     const long tiles = (long)((p.N + 127) / 128) * ((p.M + c.bn - 1) / c.bn);
     const long nkb = (p.K + c.bk - 1) / c.bk;
@@ -216,6 +217,11 @@ qgemm_config_t heuristic(const Problem &p, int sms)
         const long tiles = (long)((p.N + 31) / 32) * ((p.M + 15) / 16);
         c.split_k = pick_split(tiles, p.K / kb, 12, sms);
         if (p.gs % 128 == 0) c.stages = 4;       // TMA-fed kernel
+    } else if (p.op == QG_OP_W2A8 && p.K % 256 == 0) {
+        c.rows = 64;                               // TMA-fed tensor-core kernel
+        c.stages = 4;
+        const long tiles = (long)((p.N + 63) / 64) * ((p.M + 15) / 16);
+        c.split_k = pick_split(tiles, p.K / 256, 12, sms);
     } else {
         c.rows = 4;
         const int kc = p.op == QG_OP_W2A8 ? 64 : 16;
@@ -315,6 +321,8 @@ qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStre
         if (p.op == QG_OP_W4A16)
             e = c.stages ? launch_gemv_w4a16_tma(p, c, d->err_word, stream)
                          : launch_gemv_w4a16(p, c, stream);
+        else if (p.op == QG_OP_W2A8 && c.stages)
+            e = launch_gemv_w2a8_tma(p, c, d->err_word, stream);
         else
             e = launch_gemv_int(p, c, stream);
     } else if (c.path == QG_PATH_TC) {
@@ -356,11 +364,12 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
         c.path = QG_PATH_GEMV;
         const int rows16[] = {16, 32, 64};
         const int rows_int[] = {1, 2, 4, 8};
-        const int *rows = p.op == QG_OP_W4A16 ? rows16 : rows_int;
-        const int nrows = p.op == QG_OP_W4A16 ? 3 : 4;
+        const int rows_w2[] = {1, 2, 4, 8, 16, 32, 64};
+        const int *rows = p.op == QG_OP_W4A16 ? rows16 : (p.op == QG_OP_W2A8 ? rows_w2 : rows_int);
+        const int nrows = p.op == QG_OP_W4A16 ? 3 : (p.op == QG_OP_W2A8 ? 7 : 4);
         const int stage_opts[5] = {0, 2, 3, 4, 6};     // 0: register-prefetch kernel
         for (int r = 0; r < nrows; ++r)
-            for (int st = 0; st < (p.op == QG_OP_W4A16 ? 5 : 1); ++st)
+            for (int st = 0; st < (p.op == QG_OP_W8A8 ? 1 : 5); ++st)
                 for (int s = 1; s <= 16; s *= 2) {
                     c.rows = rows[r];
                     c.stages = stage_opts[st];

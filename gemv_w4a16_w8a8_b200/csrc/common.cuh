@@ -28,6 +28,8 @@ struct Problem {
 cudaError_t launch_gemv_w4a16(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
 cudaError_t launch_gemv_w4a16_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
                                   cudaStream_t stream);
+cudaError_t launch_gemv_w2a8_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
+                                 cudaStream_t stream);
 cudaError_t launch_gemv_int(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
 cudaError_t launch_pack_int4(const uint8_t *codes, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
@@ -39,6 +41,7 @@ cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int 
 // Whether a configuration can run the problem (tile and alignment rules of its kernel).
 bool gemv_w4a16_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &cfg);
+bool gemv_w2a8_tma_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
 bool tc_supports(const Problem &p, const qgemm_config_t &cfg);
 // Deepest pipeline (2..5) whose shared memory fits for this op and token tile.

@@ -201,7 +201,7 @@ void launch_r(const Problem &p, int rows, int split_k, cudaStream_t stream)
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg)
 {
     const int kc = p.op == QG_OP_W2A8 ? 64 : 16;
-    return p.K % kc == 0 && (cfg.rows == 1 || cfg.rows == 2 || cfg.rows == 4 || cfg.rows == 8) &&
+    return p.K % kc == 0 && cfg.stages == 0 && (cfg.rows == 1 || cfg.rows == 2 || cfg.rows == 4 || cfg.rows == 8) &&
            cfg.split_k >= 1 && cfg.split_k <= 64;
 }
 

@@ -120,32 +120,46 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
 
     // constant operand: rows 0..7 give sum c_k a_k, rows 8..15 give sum a_k
     const uint32_t kones[4] = {0x64006400u, 0x3C003C00u, 0x64006400u, 0x4C004C00u};
-    int consumed = 0;
-    for (int i = 0; i < cnt; ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(smem_u32(&full[warp][s]), (i / STAGES) & 1, abort_v, err)) break;
-        const int kb = first + kWarps * i;
-        const int k0 = kb * kKB;
-        // activations for this k-block, re-paired and odd halves scaled by 1/16
-        uint32_t b[NT][4][4];
+    // activations and scale / zero bits of k-block i are loaded during k-block i - 1
+    uint4 av[NT][4];
+    uint16_t sbits[RB][2], zbits[RB][2];
+    auto prefetch = [&](int i) {
+        const int k0 = (first + kWarps * i) * kKB;
+        const int g = k0 / gs;
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (aok[t]) v = ld_cached_v4(arow[t] + k0 + 8 * j);
-                act_pairs_scaled(v, b[t][j]);
-            }
-        const int g = k0 / gs;
-        float sc[RB][2], zr[RB][2];
+            for (int j = 0; j < 4; ++j)
+                av[t][j] = aok[t] ? ld_cached_v4(arow[t] + k0 + 8 * j) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int r = 0; r < RB; ++r)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const size_t gi = (size_t)srow[r][h] * G + g;
-                sc[r][h] = half_bits_to_float(ld_cached_u16(S + gi));
-                zr[r][h] = zero_pt ? half_bits_to_float(ld_cached_u16(Z + gi)) : 0.f;
+                sbits[r][h] = ld_cached_u16(S + gi);
+                zbits[r][h] = zero_pt ? ld_cached_u16(Z + gi) : (uint16_t)0;
             }
+    };
+    if (cnt > 0) prefetch(0);
+    int consumed = 0;
+    for (int i = 0; i < cnt; ++i) {
+        const int s = i % STAGES;
+        // take this k-block's activations and scales out of the prefetch registers
+        uint32_t b[NT][4][4];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) act_pairs_scaled(av[t][j], b[t][j]);
+        float sc[RB][2], zr[RB][2];
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sc[r][h] = half_bits_to_float(sbits[r][h]);
+                zr[r][h] = half_bits_to_float(zbits[r][h]);
+            }
+        if (i + 1 < cnt) prefetch(i + 1);
+        if (!mbar_wait(smem_u32(&full[warp][s]), (i / STAGES) & 1, abort_v, err)) break;
         float cz[NT][4];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {

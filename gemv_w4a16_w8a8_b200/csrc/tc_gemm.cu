@@ -21,6 +21,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,7 +32,7 @@ namespace {
 
 enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3 };
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
 constexpr int kSlabBytes = 128;        // bytes of K per stage and row (64 fp16 / 128 int8)
 constexpr int kGroupT = 8;             // token tiles per raster group
@@ -100,54 +101,72 @@ template <int MODE> struct Traits {
     static constexpr int c_bytes = (MODE == kDense || MODE == kW4A16) ? 2 : 4;
 };
 
+// Shared memory: a ring of STAGES TMA stages (weight slab as loaded + activation slab) and,
+// for packed weights, a separate ring of DQ buffers holding the upcast weight slab the MMA
+// reads. The upcast slab only lives from its dequantisation to its MMA, so it needs fewer
+// buffers than the TMA ring needs stages; keeping them apart leaves room for a deeper ring.
+constexpr int kMaxSmem = 227 * 1024;
+
+constexpr int smem_total(bool packed, int bn, int stages, int dq)
+{
+    return 1024 + stages * ((packed ? kRowsW * 32 : kRowsW * kSlabBytes) + bn * kSlabBytes) +
+           (packed ? dq * kRowsW * kSlabBytes : 0) + 8 * (3 * stages + 2 * dq + 5) + 16;
+}
+
+constexpr int dq_buffers(bool packed, int bn, int stages)
+{
+    return !packed ? 0 : (smem_total(true, bn, stages, 3) <= kMaxSmem ? 3 : 2);
+}
+
 template <int MODE, int BN, int STAGES> struct Smem {
+    static constexpr bool packed = Traits<MODE>::packed;
     static constexpr int w_tma = Traits<MODE>::w_tma_bytes;
-    static constexpr int w_mma = Traits<MODE>::w_mma_bytes;
     static constexpr int a_bytes = BN * kSlabBytes;
-    static constexpr int stage = w_tma + w_mma + a_bytes;
-    static constexpr int bars = 8 * (3 * STAGES + 1) + 16;
-    static constexpr int total = 1024 + STAGES * stage + bars;
+    static constexpr int stage = w_tma + a_bytes;
+    static constexpr int dq = dq_buffers(packed, BN, STAGES);
+    static constexpr int dq_bytes = kRowsW * kSlabBytes;
+    static constexpr int nbars = 3 * STAGES + 2 * dq + 5;   // ring x2, dq x2, accum x4, final
+    static constexpr int total = smem_total(packed, BN, STAGES, dq);
 };
 
-template <int BN> constexpr uint32_t tmem_cols() { return BN < 32 ? 32u : (uint32_t)BN; }
+// two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
+template <int BN> constexpr uint32_t tmem_cols() { return 2 * BN < 32 ? 32u : (uint32_t)(2 * BN); }
 
-// Upcast one 128-row slab of packed int4 (8 words per row) into fp16 (q - z) * s, written in
-// the SWIZZLE_128B K-major layout. Thread r owns weight row r of the tile.
-__device__ __forceinline__ void dequant_w4(const uint32_t *packed, uint8_t *dst, int r,
-                                           uint32_t sz0, uint32_t sz1, uint32_t nz0, uint32_t nz1)
+// Upcast half a slab of packed int4 (words 4h..4h+3 of weight row r: 32 values of K, one
+// quantisation group) into fp16 (q - z) * s = fma(q, s, fp16(-z * s)), written in the
+// SWIZZLE_128B K-major layout the MMA reads.
+__device__ __forceinline__ void dequant_w4(const uint32_t *packed, uint8_t *dst, int r, int h,
+                                           uint32_t sc, uint32_t nz)
 {
     constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
     constexpr uint32_t kInv16 = 0x2C002C00u, kNeg64 = 0xD400D400u;
-    const uint4 p0 = *reinterpret_cast<const uint4 *>(packed + r * 8);
-    const uint4 p1 = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4);
-    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    const uint4 p = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4 * (h ^ ((r >> 2) & 1)));
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         const uint32_t w = words[j], w8 = w >> 8;
         const uint32_t h0 = hsub2_u32(lop3_and_or(w, kLo, kMagic), kMagic);        // q0 q4
         const uint32_t h1 = hfma2_u32(lop3_and_or(w, kHi, kMagic), kInv16, kNeg64); // q1 q5
         const uint32_t h2 = hsub2_u32(lop3_and_or(w8, kLo, kMagic), kMagic);       // q2 q6
         const uint32_t h3 = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);// q3 q7
-        const uint32_t s = j < 4 ? sz0 : sz1, nz = j < 4 ? nz0 : nz1;
         uint4 o;
-        o.x = hfma2_u32(prmt(h0, h1, 0x5410), s, nz);   // (q0, q1)
-        o.y = hfma2_u32(prmt(h2, h3, 0x5410), s, nz);   // (q2, q3)
-        o.z = hfma2_u32(prmt(h0, h1, 0x7632), s, nz);   // (q4, q5)
-        o.w = hfma2_u32(prmt(h2, h3, 0x7632), s, nz);   // (q6, q7)
-        *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = o;
+        o.x = hfma2_u32(prmt(h0, h1, 0x5410), sc, nz);   // (q0, q1)
+        o.y = hfma2_u32(prmt(h2, h3, 0x5410), sc, nz);   // (q2, q3)
+        o.z = hfma2_u32(prmt(h0, h1, 0x7632), sc, nz);   // (q4, q5)
+        o.w = hfma2_u32(prmt(h2, h3, 0x7632), sc, nz);   // (q6, q7)
+        *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }
 }
 
-// Upcast one slab of packed int2 (8 words = 128 values per row) into int8 values -2..1.
-__device__ __forceinline__ void dequant_w2(const uint32_t *packed, uint8_t *dst, int r)
+// Upcast half a slab of packed int2 (words 4h..4h+3 of weight row r: 64 values) into int8.
+__device__ __forceinline__ void dequant_w2(const uint32_t *packed, uint8_t *dst, int r, int h)
 {
-    const uint4 p0 = *reinterpret_cast<const uint4 *>(packed + r * 8);
-    const uint4 p1 = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4);
-    const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    const uint4 p = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4 * (h ^ ((r >> 2) & 1)));
+    const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < 4; ++j) {
         const uint32_t wf = words[j] ^ 0xAAAAAAAAu;           // u' = u ^ 2, value = u' - 2
         const uint32_t f0 = wf & 0x03030303u;                 // fields 0, 4, 8, 12
         const uint32_t f1 = (wf >> 2) & 0x03030303u;          // fields 1, 5, 9, 13
@@ -166,7 +185,7 @@ __device__ __forceinline__ void dequant_w2(const uint32_t *packed, uint8_t *dst,
         o.y = (o.y + 0x7E7E7E7Eu) ^ 0x80808080u;
         o.z = (o.z + 0x7E7E7E7Eu) ^ 0x80808080u;
         o.w = (o.w + 0x7E7E7E7Eu) ^ 0x80808080u;
-        *reinterpret_cast<uint4 *>(row + ((j ^ (r & 7)) << 4)) = o;
+        *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }
 }
 
@@ -176,11 +195,42 @@ __device__ __forceinline__ uint32_t half2_bcast(float x)
     return (uint32_t)b | ((uint32_t)b << 16);
 }
 
+// Output tile of work unit u: units enumerate (split, token-tile group, weight tile, token tile).
+struct Unit {
+    int n0, t0, kb0, nk;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv, int nkb,
+                                        int kbps)
+{
+    const int tiles = n_tiles * t_tiles;
+    const int split = u / tiles;
+    const int tile = u - split * tiles;
+    const int per_group = kGroupT * n_tiles;
+    const int group = tile / per_group;
+    const int first_t = group * kGroupT;
+    const int gt = min(kGroupT, t_tiles - first_t);
+    const int within = tile - group * per_group;
+    Unit w;
+    w.t0 = (first_t + within % gt) * BNv;
+    w.n0 = (within / gt) * kRowsW;
+    w.kb0 = split * kbps;
+    w.nk = max(0, min(nkb, w.kb0 + kbps) - w.kb0);
+    return w;
+}
+
+// Persistent kernel: each CTA walks work units blockIdx.x, blockIdx.x + gridDim.x, ... The
+// shared-memory ring runs on across units, and the accumulator is double-buffered in TMEM so the
+// epilogue of one unit overlaps the main loop of the next.
+//   warps 0-3  epilogue (warp w reads TMEM lanes 32w..32w+31)
+//   warp 4     TMA producer          warp 5  TMEM allocation + MMA issue
+//   warps 8-15 dequantisation of packed weights (two threads per weight row of the tile)
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
-               int M, int N, int K, int gs, int kb_per_split, int atomic_out, unsigned int *err)
+               int M, int N, int K, int gs, int kb_per_split, int units, int atomic_out,
+               unsigned int *err)
 {
     using T = Traits<MODE>;
     using L = Smem<MODE, BN, STAGES>;
@@ -190,54 +240,49 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * L::stage);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 1);
+    uint64_t *bars =
+        reinterpret_cast<uint64_t *>(base + STAGES * L::stage + L::dq * L::dq_bytes);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + L::nbars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-
-    // tile coordinates: token-tile groups of kGroupT, weight tiles fastest inside a group
     const int n_tiles = (N + kRowsW - 1) / kRowsW;
     const int t_tiles = (M + BN - 1) / BN;
-    const int bid = blockIdx.x;
-    const int per_group = kGroupT * n_tiles;
-    const int group = bid / per_group;
-    const int first_t = group * kGroupT;
-    const int gt = min(kGroupT, t_tiles - first_t);
-    const int within = bid - group * per_group;
-    const int t_tile = first_t + within % gt;
-    const int n_tile = within / gt;
-    const int n0 = n_tile * kRowsW;
-    const int t0 = t_tile * BN;
-
     const int nkb = (K + T::k_per_slab - 1) / T::k_per_slab;
-    const int kb0 = blockIdx.y * kb_per_split;
-    const int kb1 = min(nkb, kb0 + kb_per_split);
-    if (kb0 >= kb1) return;          // empty split (C was zeroed by the host)
-    const int nk = kb1 - kb0;
 
+    constexpr int DQ = L::dq;
     auto full_bar = [&](int s) { return smem_u32(bars + s); };
-    auto deq_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
-    auto empty_bar = [&](int s) { return smem_u32(bars + 2 * STAGES + s); };
-    const uint32_t accum_bar = smem_u32(bars + 3 * STAGES);
+    auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
+    auto dqf_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + d); };
+    auto dqe_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + DQ + d); };
+    auto accf_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * DQ + b); };
+    auto acce_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * DQ + 2 + b); };
+    const uint32_t final_bar = smem_u32(bars + 2 * STAGES + 2 * DQ + 4);
     auto w_tma = [&](int s) { return base + s * L::stage; };
-    auto w_mma = [&](int s) { return base + s * L::stage + L::w_tma; };
-    auto a_tile = [&](int s) { return base + s * L::stage + L::w_tma + L::w_mma; };
+    auto a_tile = [&](int s) { return base + s * L::stage + L::w_tma; };
+    auto w_dq = [&](int d) { return base + STAGES * L::stage + d * L::dq_bytes; };
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(deq_bar(s), 128);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(accum_bar, 1);
+        for (int d = 0; d < DQ; ++d) {
+            mbar_init(dqf_bar(d), 256);
+            mbar_init(dqe_bar(d), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(accf_bar(b), 1);
+            mbar_init(acce_bar(b), 4);
+        }
+        mbar_init(final_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_proxy_async_smem();
     }
-    if (warp == 1) {
+    if (warp == 5) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_holder)),
                      "r"(kCols)
@@ -247,100 +292,164 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_d = *tmem_holder;
+    const uint32_t tmem_base = *tmem_holder;
 
-    if (warp == 0) {
+    if (warp == 4) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
             constexpr uint32_t kTx = L::w_tma + L::a_bytes;
-            const int wx_per_kb = Traits<MODE>::packed ? 8 : T::k_per_slab;   // x units of tm_w
-            int issued = 0;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1;
-                if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, err)) break;
-                mbar_expect_tx(full_bar(s), kTx);
-                const int kb = kb0 + i;
-                tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * wx_per_kb, n0);
-                tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kb * T::k_per_slab, t0);
-                ++issued;
+            const int wx_per_kb = T::packed ? 8 : T::k_per_slab;   // x units of tm_w per slab
+            int it = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                for (int i = 0; i < w.nk; ++i, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_expect_tx(full_bar(s), kTx);
+                    const int kb = w.kb0 + i;
+                    tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * wx_per_kb, w.n0);
+                    tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kb * T::k_per_slab, w.t0);
+                }
             }
-            // let every copy this thread started land before the CTA can exit
-            for (int i = max(0, issued - STAGES); i < issued; ++i) {
+            // every copy this thread started must land before the CTA can exit
+            for (int i = max(0, it - STAGES); i < it; ++i) {
                 int dummy_abort = 0;
                 mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 5) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1;
-                if (!mbar_wait(full_bar(s), ph, abort_flag, err)) break;
-                if constexpr (T::packed) {
-                    if (!mbar_wait(deq_bar(s), ph, abort_flag, err)) break;
-                }
+            int it = 0, j = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                if (w.nk == 0) continue;
+                const int b = j & 1;
+                if (!mbar_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(T::packed ? w_mma(s) : w_tma(s));
-                const uint64_t adesc = sw128_desc(a_base);
-                const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
+                const uint32_t dtm = tmem_base + (uint32_t)(b * BN);
+                for (int i = 0; i < w.nk; ++i, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(full_bar(s), ph, abort_flag, err)) {
+                        stop = true;
+                        break;
+                    }
+                    const int d = T::packed ? it % DQ : 0;
+                    if constexpr (T::packed) {
+                        if (!mbar_wait(dqf_bar(d), (it / DQ) & 1, abort_flag, err)) {
+                            stop = true;
+                            break;
+                        }
+                    }
+                    tc_fence_after();
+                    const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
+                    const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
-                    mma_issue<MODE>(tmem_d, adesc + 2 * k, bdesc + 2 * k, kIdesc,
-                                    (i | k) != 0 ? 1u : 0u);
-                mma_commit(empty_bar(s));
-            }
-            mma_commit(accum_bar);
-        }
-    } else if (warp >= 4) {
-        const int r = tid - 128;           // weight row of the tile / TMEM lane
-        // ---------------- dequantisation (packed weights) ----------------
-        if constexpr (T::packed) {
-            const int n = min(n0 + r, N - 1);
-            const int G = K / gs;
-            for (int i = 0; i < nk; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1;
-                if (!mbar_wait(full_bar(s), ph, abort_flag, err)) break;
-                const uint32_t *packed = reinterpret_cast<const uint32_t *>(w_tma(s));
-                if constexpr (MODE == kW4A16) {
-                    const int k0 = (kb0 + i) * 64;
-                    const int g0 = min(k0 / gs, G - 1), g1 = min((k0 + 32) / gs, G - 1);
-                    const float s0 = __half2float(S[(size_t)n * G + g0]);
-                    const float s1 = __half2float(S[(size_t)n * G + g1]);
-                    const float z0 = Z ? __half2float(Z[(size_t)n * G + g0]) : 0.f;
-                    const float z1 = Z ? __half2float(Z[(size_t)n * G + g1]) : 0.f;
-                    dequant_w4(packed, w_mma(s), r, half2_bcast(s0), half2_bcast(s1),
-                               half2_bcast(-z0 * s0), half2_bcast(-z1 * s1));
-                } else {
-                    dequant_w2(packed, w_mma(s), r);
+                    for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
+                        mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                        (i | k) != 0 ? 1u : 0u);
+                    mma_commit(empty_bar(s));
+                    if constexpr (T::packed) mma_commit(dqe_bar(d));
                 }
+                mma_commit(accf_bar(b));
+                ++j;
+            }
+            // nothing may still run on the tensor cores when TMEM is released
+            mma_commit(final_bar);
+            int dummy_abort = 0;
+            mbar_wait(final_bar, 0, &dummy_abort, nullptr);
+        }
+    } else if (warp >= 8) {
+        // ---------------- dequantisation (packed weights) ----------------
+        // 256 threads: thread (h, r) upcasts words 4h..4h+3 of weight row r of every slab. The
+        // scale and zero of the next slab are loaded while the current one is processed.
+        if constexpr (T::packed) {
+            const int dq = tid - 256;
+            const int r = dq & 127, h = dq >> 7;
+            const int G = K / gs;
+            int u = blockIdx.x, i = 0, it = 0;
+            Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            auto skip_empty = [&]() {
+                while (u < units && i >= w.nk) {
+                    u += gridDim.x;
+                    i = 0;
+                    if (u < units) w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                }
+            };
+            // (scale, -zero*scale) of slab i of unit w for this thread, as fp16 pairs
+            auto fetch = [&](const Unit &ww, int ii, float &sc, float &zz) {
+                const int n = min(ww.n0 + r, N - 1);
+                const int g = min(((ww.kb0 + ii) * 64 + 32 * h) / gs, G - 1);
+                sc = half_bits_to_float(ld_cached_u16(S + (size_t)n * G + g));
+                zz = Z ? half_bits_to_float(ld_cached_u16(Z + (size_t)n * G + g)) : 0.f;
+            };
+            skip_empty();
+            float sc = 0.f, zz = 0.f;
+            if (MODE == kW4A16 && u < units) fetch(w, i, sc, zz);
+            while (u < units) {
+                // position of the next slab, and its scale / zero in flight
+                int u2 = u, i2 = i + 1;
+                Unit w2 = w;
+                while (u2 < units && i2 >= w2.nk) {
+                    u2 += gridDim.x;
+                    i2 = 0;
+                    if (u2 < units) w2 = unit_of(u2, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                }
+                float sc2 = 0.f, zz2 = 0.f;
+                if (MODE == kW4A16 && u2 < units) fetch(w2, i2, sc2, zz2);
+                const int s = it % STAGES, d = it % DQ;
+                if (!mbar_wait(dqe_bar(d), ((it / DQ) & 1) ^ 1, abort_flag, err)) break;
+                if (!mbar_wait(full_bar(s), (it / STAGES) & 1, abort_flag, err)) break;
+                const uint32_t *packed = reinterpret_cast<const uint32_t *>(w_tma(s));
+                if constexpr (MODE == kW4A16)
+                    dequant_w4(packed, w_dq(d), r, h, half2_bcast(sc), half2_bcast(-zz * sc));
+                else
+                    dequant_w2(packed, w_dq(d), r, h);
                 fence_proxy_async_smem();
-                mbar_arrive(deq_bar(s));
+                mbar_arrive(dqf_bar(d));
+                ++it;
+                u = u2;
+                i = i2;
+                w = w2;
+                sc = sc2;
+                zz = zz2;
             }
         }
+    } else if (warp < 4) {
         // ---------------- epilogue ----------------
-        bool ok = mbar_wait(accum_bar, 0, abort_flag, err);
-        tc_fence_after();
-        // tcgen05.ld is warp-collective: decide per warp, never per lane
-        ok = __all_sync(0xffffffffu, ok && !*abort_flag);
-        if (ok) {
-            const int n = n0 + r;
-            const uint32_t lane_addr = tmem_d + ((uint32_t)((warp - 4) * 32) << 16);
-            // fp16 results leave as (n, n+1) pairs: rows n and n+1 sit in neighbouring lanes
-            const bool pairs = (N & 1) == 0;
+        const int r = tid;                                 // weight row of the tile = TMEM lane
+        const bool pairs = (N & 1) == 0;
+        int j = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            if (w.nk == 0) continue;
+            const int b = j & 1;
+            bool ok = mbar_wait(accf_bar(b), (j >> 1) & 1, abort_flag, err);
+            tc_fence_after();
+            // tcgen05.ld is warp-collective: decide per warp, never per lane
+            ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+            if (!ok) break;
+            const int n = w.n0 + r;
+            const uint32_t lane_addr =
+                tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
 #pragma unroll 1
             for (int c = 0; c < BN; c += 16) {
-                if (t0 + c >= M) break;
+                if (w.t0 + c >= M) break;
                 uint32_t v[16];
                 tmem_ld16(lane_addr + c, v);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = t0 + c + j;         // the same in every lane
+                for (int e = 0; e < 16; ++e) {
+                    const int t = w.t0 + c + e;           // the same in every lane
                     if (t >= M) break;
                     if constexpr (T::c_bytes == 2) {
-                        const float x = __uint_as_float(v[j]);
+                        // fp16 results leave as (n, n+1) pairs from neighbouring lanes
+                        const float x = __uint_as_float(v[e]);
                         const float y = __shfl_xor_sync(0xffffffffu, x, 1);
                         __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
                         if (pairs) {
@@ -355,19 +464,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         }
                     } else if (n < N) {
                         int32_t *dst = static_cast<int32_t *>(C) + (size_t)t * N + n;
-                        if (atomic_out) red_add_s32(dst, (int)v[j]);
-                        else *dst = (int)v[j];
+                        if (atomic_out) red_add_s32(dst, (int)v[e]);
+                        else *dst = (int)v[e];
                     }
                 }
             }
+            // this warp is done with accumulator buffer b
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce_bar(b));
+            ++j;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 5) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d),
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(kCols)
                      : "memory");
     }
@@ -388,12 +502,8 @@ int mode_of(int op)
 int smem_bytes(int mode, int bn, int stages)
 {
     const bool packed = (mode == kW4A16 || mode == kW2A8);
-    const int stage = (packed ? kRowsW * 32 + kRowsW * kSlabBytes : kRowsW * kSlabBytes) +
-                      bn * kSlabBytes;
-    return 1024 + stages * stage + 8 * (3 * stages + 1) + 16;
+    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages));
 }
-
-constexpr int kMaxSmem = 227 * 1024;
 
 template <int MODE, int BN, int STAGES>
 cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
@@ -431,12 +541,12 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                       CU_TENSOR_MAP_SWIZZLE_128B);
     } else if constexpr (MODE == kW4A16) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
-                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_32B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
                       BN, CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 16, p.N, (uint64_t)p.K / 4,
-                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_32B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     }
@@ -447,11 +557,27 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     const int splits = (nkb + kbps - 1) / kbps;
     const int n_tiles = (p.N + kRowsW - 1) / kRowsW;
     const int t_tiles = (p.M + BN - 1) / BN;
-    dim3 grid(n_tiles * t_tiles, splits);
+    const long units = (long)n_tiles * t_tiles * splits;
+    if (units > 0x7fffffffL) return cudaErrorInvalidValue;
+    // persistent grid: as many CTAs as fit on the device at once (shared memory, threads and
+    // the TMEM columns each CTA holds), never more than there are units
+    static int per_sm[64] = {};
+    static int sm_count[64] = {};
+    if (!per_sm[dev]) {
+        int occ = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::total) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return cudaErrorInvalidConfiguration;
+        occ = std::min(occ, (int)(512 / tmem_cols<BN>()));
+        sm_count[dev] = sms;
+        per_sm[dev] = std::max(1, occ);
+    }
+    const int grid = (int)std::min<long>(units, (long)per_sm[dev] * sm_count[dev]);
     kern<<<grid, kThreads, L::total, stream>>>(
         tw, ta, static_cast<const __half *>(p.scales),
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, p.C, p.M, p.N, p.K, p.gs,
-        kbps, split_k > 1 ? 1 : 0, err);
+        kbps, (int)units, split_k > 1 ? 1 : 0, err);
     return cudaGetLastError();
 }
 

@@ -175,8 +175,9 @@ def test_tc_split_fills_the_gpu():
 
 def test_tc_config_limits():
     M, N, K = 256, 512, 1024
-    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 4))      # 214 KB of smem
-    for bad in (_tc(256, 5), _tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
+    # packed weights: 5 TMA stages of 36 KB plus two 16 KB dequant buffers fit (213 KB)
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 5))
+    for bad in (_tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
         with pytest.raises(qg.QGemmError):
             qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, bad)
     qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 4))

@@ -89,3 +89,19 @@ def test_int_guard_bands(op):
     torch.cuda.synchronize()
     assert guards_intact(buf, pad, 3 * 130)
     assert np.array_equal(C.cpu().numpy(), case.ref_full())
+
+
+@pytest.mark.parametrize("rows", [16, 32, 64])
+@pytest.mark.parametrize("stages", [2, 3, 4, 6])
+@pytest.mark.parametrize("M", [1, 7, 16])
+def test_w2a8_tma_kernel_configs(rows, stages, M):
+    N, K = 200, 4096
+    case = IntCase("w2a8", M, N, K, seed=rows + stages + M)
+    for split in (1, 3):
+        cfg = {"path": qg.PATH_GEMV, "rows": rows, "bm": 0, "bn": 0, "bk": 0, "stages": stages,
+               "split_k": split, "swap_ab": 0}
+        qg.qgemm_set_config(qg.OP_W2A8, M, N, K, -1, 0, cfg)
+        try:
+            assert np.array_equal(case.run().cpu().numpy(), case.ref_full()), (rows, stages, split)
+        finally:
+            qg.qgemm_set_config(qg.OP_W2A8, M, N, K, -1, 0, None)
