@@ -32,7 +32,7 @@ PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 
 # every symbol include/qgemm.h declares
 EXPORTS = (
-    "qgemm_w4a16", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "qgemm_w4a16", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
     "qgemm_version",
@@ -68,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, i32 = ctypes.c_void_p, ctypes.c_int
         L.qgemm_w4a16.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.qgemm_w4a16_splitk_f32.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                             ctypes.c_size_t, vp]
+        L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.qgemm_w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_w2a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_dense_f16.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
@@ -86,7 +90,8 @@ def lib() -> ctypes.CDLL:
         L.qgemm_status_string.restype = ctypes.c_char_p
         L.qgemm_version.restype = i32
         for name in EXPORTS:
-            if name not in ("qgemm_status_string", "qgemm_clear_configs", "qgemm_version"):
+            if name not in ("qgemm_status_string", "qgemm_clear_configs", "qgemm_version",
+                            "qgemm_w4a16_workspace_bytes"):
                 getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -153,6 +158,36 @@ def qgemm_w4a16(A, Wq, scales, zeros=None, C=None, group_size: int = 128, split_
     st = lib().qgemm_w4a16(_ptr(A), _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(C), M, N, K,
                            group_size, split_k, int(zeros is not None), _stream(stream))
     _check(st, "qgemm_w4a16")
+    return C
+
+
+def qgemm_w4a16_workspace_bytes(M: int, N: int, K: int, group_size: int, split_k: int) -> int:
+    return int(lib().qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k))
+
+
+def qgemm_w4a16_splitk_f32(A, Wq, scales, zeros=None, C=None, group_size: int = 128,
+                           split_k: int = 4, workspace=None, stream=None):
+    """Deterministic split-K W4A16 through an fp32 workspace (a uint8 CUDA tensor of at least
+    qgemm_w4a16_workspace_bytes(...) bytes; allocated here when not given)."""
+    torch = _torch()
+    _need(A, torch.float16, 2, "A")
+    _need(Wq, (torch.int32, torch.uint32), 2, "Wq")
+    _need(scales, torch.float16, 2, "scales")
+    if zeros is not None:
+        _need(zeros, torch.float16, 2, "zeros")
+    M, K = A.shape
+    N = Wq.shape[0]
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _need(C, torch.float16, 2, "C")
+    need = qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=A.device)
+    _need(workspace, torch.uint8, 1, "workspace")
+    st = lib().qgemm_w4a16_splitk_f32(_ptr(A), _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(C), M, N,
+                                      K, group_size, split_k, int(zeros is not None),
+                                      _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "qgemm_w4a16_splitk_f32")
     return C
 
 

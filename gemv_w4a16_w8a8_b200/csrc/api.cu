@@ -190,7 +190,11 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     c.bm = 128;
     c.bn = pow2_at_least(p.M, 16, 256);
     c.bk = k_per_slab(p.op);
+    // packed weights: the deepest ring that still leaves three dequant buffers (measured faster
+    // than one more TMA stage with two); other ops: the deepest ring that fits
     c.stages = tc_max_stages(p.op, c.bn);
+    if ((p.op == QG_OP_W4A16 || p.op == QG_OP_W2A8) && c.stages > 2 && tc_dq_buffers(p.op, c.bn, c.stages) < 3)
+        --c.stages;
     c.swap_ab = 1;
     const long tiles = (long)((p.N + 127) / 128) * ((p.M + c.bn - 1) / c.bn);
     const long nkb = (p.K + c.bk - 1) / c.bk;
@@ -410,6 +414,65 @@ qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, con
 {
     return matmul(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, split_k, has_zero,
                   stream);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// counters: one per output tile of the smallest row tile (16) and token tile (8) the streaming
+// kernel uses, so the bound holds for every configuration; partials: split_k planes of M x N fp32
+static size_t ws_counter_bytes(int M, int N)
+{
+    return align256((size_t)((N + 15) / 16) * (size_t)((M + 7) / 8) * sizeof(unsigned int));
+}
+
+size_t qgemm_w4a16_workspace_bytes(int M, int N, int K, int group_size, int split_k)
+{
+    if (check_shape(QG_OP_W4A16, M, N, K, group_size, 0, split_k) != QG_OK || split_k < 1)
+        return 0;
+    return ws_counter_bytes(M, N) + (size_t)split_k * M * N * sizeof(float);
+}
+
+qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *scales,
+                                 const void *zeros, void *C, int M, int N, int K, int group_size,
+                                 int split_k, int has_zero, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream)
+{
+    qg_status s = check_shape(QG_OP_W4A16, M, N, K, group_size, has_zero, split_k);
+    if (s != QG_OK) return s;
+    if (split_k < 1) return QG_ERR_INVALID_ARG;
+    if (effective_gs(QG_OP_W4A16, K, group_size) % 128) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!A || !Wq || !C || !scales || !workspace) return QG_ERR_INVALID_ARG;
+    if ((zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(Wq, 16) || !aligned(C, 16) || !aligned(workspace, 256) ||
+        !aligned(scales, 2) || (zeros && !aligned(zeros, 2)))
+        return QG_ERR_ALIGNMENT;
+    if (workspace_bytes < qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k))
+        return QG_ERR_INVALID_ARG;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    Problem p = make_problem(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, has_zero);
+    qgemm_config_t c = choose(p, split_k, d->sms);
+    if (c.path != QG_PATH_GEMV || c.stages == 0) {   // this form lives in the TMA-fed kernel
+        std::memset(&c, 0, sizeof(c));
+        c.path = QG_PATH_GEMV;
+        c.rows = 32;
+        c.stages = 4;
+    }
+    c.split_k = split_k;
+    if (!gemv_w4a16_tma_supports(p, c)) return QG_ERR_BAD_CONFIG;
+    unsigned int *counters = static_cast<unsigned int *>(workspace);
+    float *parts = reinterpret_cast<float *>(static_cast<char *>(workspace) + ws_counter_bytes(M, N));
+    if (cudaMemsetAsync(counters, 0, gemv_w4a16_ws_tiles(p, c) * sizeof(unsigned int), stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    if (launch_gemv_w4a16_tma(p, c, d->err_word, stream, parts, counters) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
 }
 
 qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N, int K,

@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/qgemm.h"
+#include "qgemm.h"
 
 namespace qg {
 
@@ -22,17 +22,25 @@ struct Problem {
     int M, N, K;
     int gs;        // effective group size (K when the caller passed -1 / 0)
     int has_zero;
+    int interleaved = 0;   // W4A16: 1 = codes of each word in nibble order 0,2,4,6,1,3,5,7
 };
 
 // Launchers return cudaGetLastError() after queueing their kernels on `stream`.
 cudaError_t launch_gemv_w4a16(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
+// ws_part / ws_count non-null: deterministic split-K through an fp32 workspace (see the
+// kernel); null: plain store or red.global.add into a zeroed C.
 cudaError_t launch_gemv_w4a16_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
-                                  cudaStream_t stream);
+                                  cudaStream_t stream, float *ws_part = nullptr,
+                                  unsigned int *ws_count = nullptr);
+// Arrival counters the deterministic split-K needs (one per output tile of this config).
+size_t gemv_w4a16_ws_tiles(const Problem &p, const qgemm_config_t &cfg);
 cudaError_t launch_gemv_w2a8_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
                                  cudaStream_t stream);
 cudaError_t launch_gemv_int(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
 cudaError_t launch_pack_int4(const uint8_t *codes, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
+cudaError_t launch_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int N, int K,
+                                         cudaStream_t stream);
 cudaError_t launch_pack_int2(const int8_t *vals, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
 cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int *err_word,
@@ -46,6 +54,8 @@ bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
 bool tc_supports(const Problem &p, const qgemm_config_t &cfg);
 // Deepest pipeline (2..5) whose shared memory fits for this op and token tile.
 int tc_max_stages(int op, int bn);
+// Number of upcast-weight buffers the tensor-core kernel keeps for this ring depth (0: none).
+int tc_dq_buffers(int op, int bn, int stages);
 
 // ------------------------------------------------------------------------------------------
 // PTX wrappers

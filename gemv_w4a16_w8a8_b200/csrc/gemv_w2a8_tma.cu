@@ -104,16 +104,17 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
         aok[t] = tok < M;
         arow[t] = A + (size_t)min(tok, M - 1) * K + 64 * lt;   // thread lt: words 4lt..4lt+3
     }
-    int acc[RB][NT][4];
-    int asum[NT][4];
+    // two independent accumulation chains per product keep the MMA pipe busy
+    int acc[RB][NT][4], acc2[RB][NT][4];
+    int asum[NT][4], asum2[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) asum[t][e] = 0;
+        for (int e = 0; e < 4; ++e) asum[t][e] = asum2[t][e] = 0;
 #pragma unroll
         for (int r = 0; r < RB; ++r)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[r][t][e] = 0;
+            for (int e = 0; e < 4; ++e) acc[r][t][e] = acc2[r][t][e] = 0;
     }
     const uint32_t kOnes[4] = {0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u};
 
@@ -132,7 +133,7 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
                 if (aok[t]) v = ld_cached_v4(arow[t] + k0 + 16 * q);
                 gather4(v, b[t][q]);
                 mma_16832_u8s8(asum[t], kOnes, b[t][q][0], b[t][q][1]);
-                mma_16832_u8s8(asum[t], kOnes, b[t][q][2], b[t][q][3]);
+                mma_16832_u8s8(asum2[t], kOnes, b[t][q][2], b[t][q][3]);
             }
         const uint8_t *slot = &ring[warp][s][0];
 #pragma unroll
@@ -152,7 +153,7 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     mma_16832_u8s8(acc[r][t], a0, b[t][q][0], b[t][q][1]);
-                    mma_16832_u8s8(acc[r][t], a1, b[t][q][2], b[t][q][3]);
+                    mma_16832_u8s8(acc2[r][t], a1, b[t][q][2], b[t][q][3]);
                 }
             }
         }
@@ -170,6 +171,14 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
     }
 
     // C = sum a u' - 2 sum a; fragment: e0 (row g, tok 2t) e1 (row g, 2t+1) e2/e3 (row g+8)
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            asum[t][e] += asum2[t][e];
+#pragma unroll
+            for (int r = 0; r < RB; ++r) acc[r][t][e] += acc2[r][t][e];
+        }
 #pragma unroll
     for (int r = 0; r < RB; ++r)
 #pragma unroll

@@ -56,18 +56,25 @@ __device__ __forceinline__ void upcast_word(uint32_t w, uint32_t (&h)[4])
     h[3] = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);
 }
 
-// Eight activations (h0..h7) re-paired to match upcast_word: (h0,h4) (h1,h5) (h2,h6) (h3,h7).
+// Eight activations (h0..h7) paired to match upcast_word: (h0,h4) (h1,h5) (h2,h6) (h3,h7) for
+// the natural packing; for the interleaved packing upcast_word yields (q0,q1) (q2,q3) (q4,q5)
+// (q6,q7), so the activations stay in natural pairs and need no permutation.
+template <bool ILV>
 __device__ __forceinline__ void act_pairs(const uint4 &v, uint32_t (&b)[4])
 {
-    b[0] = prmt(v.x, v.z, 0x5410);
-    b[1] = prmt(v.x, v.z, 0x7632);
-    b[2] = prmt(v.y, v.w, 0x5410);
-    b[3] = prmt(v.y, v.w, 0x7632);
+    if constexpr (ILV) {
+        b[0] = v.x; b[1] = v.y; b[2] = v.z; b[3] = v.w;
+    } else {
+        b[0] = prmt(v.x, v.z, 0x5410);
+        b[1] = prmt(v.x, v.z, 0x7632);
+        b[2] = prmt(v.y, v.w, 0x5410);
+        b[3] = prmt(v.y, v.w, 0x7632);
+    }
 }
 
 // WPT: packed words per thread per row per k-block (k-block = 32*WPT values of K).
 // RB:  16-row blocks per warp.  NT: 8-token tiles per CTA.
-template <int WPT, int RB, int NT>
+template <int WPT, int RB, int NT, bool ILV>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_w4a16_kernel(const __half *__restrict__ A, const uint32_t *__restrict__ Wq,
                   const __half *__restrict__ S, const __half *__restrict__ Z,
@@ -144,7 +151,7 @@ gemv_w4a16_kernel(const __half *__restrict__ A, const uint32_t *__restrict__ Wq,
             for (int j = 0; j < WPT; ++j) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (aok[t]) v = ld_cached_v4(arow[t] + (size_t)kb * KB + 8 * j);
-                act_pairs(v, b[t][j]);
+                act_pairs<ILV>(v, b[t][j]);
             }
         const int g = (kb * KB) / gs;
         float s[RB][2], z[RB][2];
@@ -265,9 +272,15 @@ gemv_w4a16_kernel(const __half *__restrict__ A, const uint32_t *__restrict__ Wq,
     }
 }
 
+template <int WPT, int RB, int NT, bool ILV>
+void launch_ilv(const Problem &p, int split_k, cudaStream_t stream);
+
 template <int WPT, int RB, int NT>
 void launch_one(const Problem &p, int split_k, cudaStream_t stream)
 {
+    if (p.interleaved) launch_ilv<WPT, RB, NT, true>(p, split_k, stream);
+    else launch_ilv<WPT, RB, NT, false>(p, split_k, stream);
+}
     constexpr int KB = 32 * WPT;
     const int nkb = p.K / KB;
     const int kbps = (nkb + split_k - 1) / split_k;

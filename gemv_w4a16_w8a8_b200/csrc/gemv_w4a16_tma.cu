@@ -50,7 +50,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__restrict__ A,
                       const __half *__restrict__ S, const __half *__restrict__ Z,
                       __half *__restrict__ C, int M, int N, int K, int gs, int kb_per_split,
-                      int atomic_out, unsigned int *err)
+                      int atomic_out, unsigned int *err, float *__restrict__ ws_part,
+                      unsigned int *__restrict__ ws_count)
 {
     using L = Layout<RB, NT, STAGES>;
     constexpr int kRows = L::rows, kSlot = L::slot, TT = L::tt, TR = L::tr;
@@ -59,6 +60,7 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
     auto full = reinterpret_cast<uint64_t (*)[STAGES]>(dsmem + L::ring_bytes);
     auto red = reinterpret_cast<float (*)[TT][TR + 1]>(dsmem + L::ring_bytes + L::bar_bytes);
     int &abort_flag = *reinterpret_cast<int *>(dsmem + L::ring_bytes + L::bar_bytes + L::red_bytes);
+    int &last_flag = *(&abort_flag + 1);
 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -160,16 +162,19 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
             }
         if (i + 1 < cnt) prefetch(i + 1);
         if (!mbar_wait(smem_u32(&full[warp][s]), (i / STAGES) & 1, abort_v, err)) break;
-        float cz[NT][4];
+        // two independent accumulation chains per product keep the MMA pipe busy
+        float cz[NT][4], cz2[NT][4];
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cz[t][e] = 0.f;
+            for (int e = 0; e < 4; ++e) cz[t][e] = cz2[t][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 mma_16816_f16(cz[t], kones, b[t][j][0], b[t][j][1], cz[t]);
-                mma_16816_f16(cz[t], kones, b[t][j][2], b[t][j][3], cz[t]);
+                mma_16816_f16(cz2[t], kones, b[t][j][2], b[t][j][3], cz2[t]);
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cz[t][e] += cz2[t][e];
         }
         const uint8_t *slot = &ring[warp][s][0];
 #pragma unroll
@@ -179,11 +184,11 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
                 *reinterpret_cast<const uint4 *>(slot + (16 * r + lg + 8) * 64 + 16 * lt);
             const uint32_t wva[4] = {wa.x, wa.y, wa.z, wa.w};
             const uint32_t wvb[4] = {wb.x, wb.y, wb.z, wb.w};
-            float d[NT][4];
+            float d[NT][4], d2[NT][4];
 #pragma unroll
             for (int t = 0; t < NT; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) d[t][e] = 0.f;
+                for (int e = 0; e < 4; ++e) d[t][e] = d2[t][e] = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
@@ -196,9 +201,13 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     mma_16816_f16(d[t], a0, b[t][j][0], b[t][j][1], d[t]);
-                    mma_16816_f16(d[t], a1, b[t][j][2], b[t][j][3], d[t]);
+                    mma_16816_f16(d2[t], a1, b[t][j][2], b[t][j][3], d2[t]);
                 }
             }
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) d[t][e] += d2[t][e];
             // d0 (row g, tok 2t) d1 (row g, tok 2t+1) d2 (row g+8, tok 2t) d3 (row g+8, 2t+1)
             // cz0/cz1: corr of tok 2t / 2t+1;  cz2/cz3: sum a of tok 2t / 2t+1
 #pragma unroll
@@ -236,6 +245,39 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
         }
     __syncthreads();
     if (abort_flag) return;
+    if (ws_part) {
+        // Deterministic split-K: park this part's fp32 tile in workspace plane blockIdx.y; the
+        // last part to finish the tile sums all planes in part order and writes fp16 C.
+        const int splits = gridDim.y;
+        for (int e = threadIdx.x; e < TT * TR; e += kWarps * 32) {
+            const int tt = e / TR, rr = e % TR;
+            const int tok = tok0 + tt, row = n0 + rr;
+            if (tok >= M || row >= N) continue;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) v += red[w][tt][rr];
+            ws_part[((size_t)blockIdx.y * M + tok) * N + row] = v;
+        }
+        __threadfence();
+        __syncthreads();
+        const unsigned int tile = blockIdx.z * gridDim.x + blockIdx.x;
+        if (threadIdx.x == 0)
+            last_flag = atomicAdd(&ws_count[tile], 1u) == (unsigned int)(splits - 1);
+        __syncthreads();
+        if (!last_flag) return;
+        __threadfence();
+        for (int e = threadIdx.x; e < TT * TR; e += kWarps * 32) {
+            const int tt = e / TR, rr = e % TR;
+            const int tok = tok0 + tt, row = n0 + rr;
+            if (tok >= M || row >= N) continue;
+            float v = 0.f;
+            for (int sp = 0; sp < splits; ++sp)
+                v += __ldcg(ws_part + ((size_t)sp * M + tok) * N + row);
+            C[(size_t)tok * N + row] = __float2half_rn(v);
+        }
+        if (threadIdx.x == 0) ws_count[tile] = 0u;   // leave the counter ready for reuse
+        return;
+    }
     const bool pairs = (N & 1) == 0;
     for (int e = threadIdx.x; e < TT * (TR / 2); e += kWarps * 32) {
         const int tt = e / (TR / 2);
@@ -266,7 +308,8 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
 }
 
 template <int RB, int NT, int STAGES>
-cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
+cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
+                       float *ws_part, unsigned int *ws_count)
 {
     using L = Layout<RB, NT, STAGES>;
     auto kern = gemv_w4a16_tma_kernel<RB, NT, STAGES>;
@@ -294,29 +337,29 @@ cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStr
     kern<<<grid, kWarps * 32, L::total, stream>>>(
         tw, static_cast<const __half *>(p.A), static_cast<const __half *>(p.scales),
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, static_cast<__half *>(p.C),
-        p.M, p.N, p.K, p.gs, kbps, split_k > 1 ? 1 : 0, err);
+        p.M, p.N, p.K, p.gs, kbps, (split_k > 1 && !ws_part) ? 1 : 0, err, ws_part, ws_count);
     return cudaGetLastError();
 }
 
 template <int RB, int NT>
 cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned int *err,
-                          cudaStream_t stream)
+                          cudaStream_t stream, float *wp, unsigned int *wc)
 {
     switch (c.stages) {
-    case 2: return launch_one<RB, NT, 2>(p, c.split_k, err, stream);
-    case 3: return launch_one<RB, NT, 3>(p, c.split_k, err, stream);
-    case 4: return launch_one<RB, NT, 4>(p, c.split_k, err, stream);
-    default: return launch_one<RB, NT, 6>(p, c.split_k, err, stream);
+    case 2: return launch_one<RB, NT, 2>(p, c.split_k, err, stream, wp, wc);
+    case 3: return launch_one<RB, NT, 3>(p, c.split_k, err, stream, wp, wc);
+    case 4: return launch_one<RB, NT, 4>(p, c.split_k, err, stream, wp, wc);
+    default: return launch_one<RB, NT, 6>(p, c.split_k, err, stream, wp, wc);
     }
 }
 
 template <int NT>
 cudaError_t launch_rb(const Problem &p, const qgemm_config_t &c, unsigned int *err,
-                      cudaStream_t stream)
+                      cudaStream_t stream, float *wp, unsigned int *wc)
 {
-    if (c.rows == 16) return launch_stages<1, NT>(p, c, err, stream);
-    if (c.rows == 32) return launch_stages<2, NT>(p, c, err, stream);
-    return launch_stages<4, NT>(p, c, err, stream);
+    if (c.rows == 16) return launch_stages<1, NT>(p, c, err, stream, wp, wc);
+    if (c.rows == 32) return launch_stages<2, NT>(p, c, err, stream, wp, wc);
+    return launch_stages<4, NT>(p, c, err, stream, wp, wc);
 }
 
 } // namespace
@@ -329,10 +372,16 @@ bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &c)
 }
 
 cudaError_t launch_gemv_w4a16_tma(const Problem &p, const qgemm_config_t &c, unsigned int *err,
-                                  cudaStream_t stream)
+                                  cudaStream_t stream, float *ws_part, unsigned int *ws_count)
 {
-    if (p.M <= 8) return launch_rb<1>(p, c, err, stream);
-    return launch_rb<2>(p, c, err, stream);
+    if (p.M <= 8) return launch_rb<1>(p, c, err, stream, ws_part, ws_count);
+    return launch_rb<2>(p, c, err, stream, ws_part, ws_count);
+}
+
+size_t gemv_w4a16_ws_tiles(const Problem &p, const qgemm_config_t &c)
+{
+    const int tt = p.M <= 8 ? 8 : 16;
+    return (size_t)((p.N + c.rows - 1) / c.rows) * (size_t)((p.M + tt - 1) / tt);
 }
 
 } // namespace qg

@@ -39,6 +39,23 @@ __global__ void pack_int4_kernel(const uint8_t *__restrict__ codes, uint32_t *__
     }
 }
 
+// interleaved layout: the even codes of a word fill its low 16 bits, the odd codes its high 16
+__global__ void pack_int4_interleaved_kernel(const uint8_t *__restrict__ codes,
+                                             uint32_t *__restrict__ packed, size_t units)
+{
+    for (size_t u = blockIdx.x * (size_t)blockDim.x + threadIdx.x; u < units;
+         u += (size_t)gridDim.x * blockDim.x) {
+        const uint4 a = ld_stream_v4(codes + 32 * u);
+        const uint4 b = ld_stream_v4(codes + 32 * u + 16);
+        const uint32_t lo[4] = {a.x, a.z, b.x, b.z}, hi[4] = {a.y, a.w, b.y, b.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            o[q] = nibbles4(prmt(lo[q], hi[q], 0x6420)) | (nibbles4(prmt(lo[q], hi[q], 0x7531)) << 16);
+        reinterpret_cast<uint4 *>(packed)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 __global__ void pack_int2_kernel(const int8_t *__restrict__ vals, uint32_t *__restrict__ packed,
                                  size_t units)
 {
@@ -69,6 +86,14 @@ cudaError_t launch_pack_int4(const uint8_t *codes, uint32_t *packed, int N, int 
 {
     const size_t units = (size_t)N * K / 32;   // K % 32 == 0 keeps units inside rows
     pack_int4_kernel<<<grid_for(units), 256, 0, stream>>>(codes, packed, units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int N, int K,
+                                         cudaStream_t stream)
+{
+    const size_t units = (size_t)N * K / 32;
+    pack_int4_interleaved_kernel<<<grid_for(units), 256, 0, stream>>>(codes, packed, units);
     return cudaGetLastError();
 }
 

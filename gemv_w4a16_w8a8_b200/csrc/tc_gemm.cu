@@ -101,16 +101,22 @@ template <int MODE> struct Traits {
     static constexpr int c_bytes = (MODE == kDense || MODE == kW4A16) ? 2 : 4;
 };
 
-// Shared memory: a ring of STAGES TMA stages (weight slab as loaded + activation slab) and,
-// for packed weights, a separate ring of DQ buffers holding the upcast weight slab the MMA
-// reads. The upcast slab only lives from its dequantisation to its MMA, so it needs fewer
-// buffers than the TMA ring needs stages; keeping them apart leaves room for a deeper ring.
+// Shared memory.
+//   dense / int8 weights: one ring of STAGES stages, each a weight slab and an activation slab
+//     loaded by TMA (SWIZZLE_128B) and read by the MMA.
+//   packed weights: three rings, so that no latency of one step sits in the cycle of another:
+//     STAGES activation slabs (TMA -> MMA), kPackedStages packed weight slabs (TMA -> upcast;
+//     4 KB each, so the upcast can run far ahead) and DQ upcast weight slabs (upcast -> MMA).
 constexpr int kMaxSmem = 227 * 1024;
+constexpr int kPackedStages = 12;
 
 constexpr int smem_total(bool packed, int bn, int stages, int dq)
 {
-    return 1024 + stages * ((packed ? kRowsW * 32 : kRowsW * kSlabBytes) + bn * kSlabBytes) +
-           (packed ? dq * kRowsW * kSlabBytes : 0) + 8 * (3 * stages + 2 * dq + 5) + 16;
+    return packed ? 1024 + stages * bn * kSlabBytes + kPackedStages * kRowsW * 32 +
+                        dq * kRowsW * kSlabBytes +
+                        8 * (2 * stages + 2 * kPackedStages + 2 * dq + 5) + 16
+                  : 1024 + stages * (kRowsW * kSlabBytes + bn * kSlabBytes) + 8 * (2 * stages + 5) +
+                        16;
 }
 
 constexpr int dq_buffers(bool packed, int bn, int stages)
@@ -120,27 +126,32 @@ constexpr int dq_buffers(bool packed, int bn, int stages)
 
 template <int MODE, int BN, int STAGES> struct Smem {
     static constexpr bool packed = Traits<MODE>::packed;
-    static constexpr int w_tma = Traits<MODE>::w_tma_bytes;
     static constexpr int a_bytes = BN * kSlabBytes;
-    static constexpr int stage = w_tma + a_bytes;
+    static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
+    static constexpr int pw_bytes = kRowsW * 32;                 // packed weight slab
+    static constexpr int sp = packed ? kPackedStages : 0;
     static constexpr int dq = dq_buffers(packed, BN, STAGES);
     static constexpr int dq_bytes = kRowsW * kSlabBytes;
-    static constexpr int nbars = 3 * STAGES + 2 * dq + 5;   // ring x2, dq x2, accum x4, final
+    // byte offsets from the 1024-aligned base
+    static constexpr int ring_bytes = packed ? STAGES * a_bytes : STAGES * (w_bytes + a_bytes);
+    static constexpr int pw_off = ring_bytes;
+    static constexpr int dq_off = pw_off + sp * pw_bytes;
+    static constexpr int bar_off = dq_off + dq * dq_bytes;
+    static constexpr int nbars = 2 * STAGES + 2 * sp + 2 * dq + 5;
     static constexpr int total = smem_total(packed, BN, STAGES, dq);
 };
 
 // two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
 template <int BN> constexpr uint32_t tmem_cols() { return 2 * BN < 32 ? 32u : (uint32_t)(2 * BN); }
 
-// Upcast half a slab of packed int4 (words 4h..4h+3 of weight row r: 32 values of K, one
+// Upcast half a slab of packed int4 (p = words 4h..4h+3 of weight row r: 32 values of K, one
 // quantisation group) into fp16 (q - z) * s = fma(q, s, fp16(-z * s)), written in the
 // SWIZZLE_128B K-major layout the MMA reads.
-__device__ __forceinline__ void dequant_w4(const uint32_t *packed, uint8_t *dst, int r, int h,
+__device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, int h,
                                            uint32_t sc, uint32_t nz)
 {
     constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
     constexpr uint32_t kInv16 = 0x2C002C00u, kNeg64 = 0xD400D400u;
-    const uint4 p = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4 * (h ^ ((r >> 2) & 1)));
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
@@ -159,10 +170,9 @@ __device__ __forceinline__ void dequant_w4(const uint32_t *packed, uint8_t *dst,
     }
 }
 
-// Upcast half a slab of packed int2 (words 4h..4h+3 of weight row r: 64 values) into int8.
-__device__ __forceinline__ void dequant_w2(const uint32_t *packed, uint8_t *dst, int r, int h)
+// Upcast half a slab of packed int2 (p = words 4h..4h+3 of weight row r: 64 values) into int8.
+__device__ __forceinline__ void dequant_w2(const uint4 &p, uint8_t *dst, int r, int h)
 {
-    const uint4 p = *reinterpret_cast<const uint4 *>(packed + r * 8 + 4 * (h ^ ((r >> 2) & 1)));
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
@@ -224,6 +234,7 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
 // epilogue of one unit overlaps the main loop of the next.
 //   warps 0-3  epilogue (warp w reads TMEM lanes 32w..32w+31)
 //   warp 4     TMA producer          warp 5  TMEM allocation + MMA issue
+//   warp 6     TMA producer of packed weight slabs (packed formats)
 //   warps 8-15 dequantisation of packed weights (two threads per weight row of the tile)
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -240,8 +251,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *bars =
-        reinterpret_cast<uint64_t *>(base + STAGES * L::stage + L::dq * L::dq_bytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bar_off);
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + L::nbars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
@@ -252,22 +262,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int t_tiles = (M + BN - 1) / BN;
     const int nkb = (K + T::k_per_slab - 1) / T::k_per_slab;
 
-    constexpr int DQ = L::dq;
+    constexpr int DQ = L::dq, SP = L::sp;
     auto full_bar = [&](int s) { return smem_u32(bars + s); };
     auto empty_bar = [&](int s) { return smem_u32(bars + STAGES + s); };
-    auto dqf_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + d); };
-    auto dqe_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + DQ + d); };
-    auto accf_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * DQ + b); };
-    auto acce_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * DQ + 2 + b); };
-    const uint32_t final_bar = smem_u32(bars + 2 * STAGES + 2 * DQ + 4);
-    auto w_tma = [&](int s) { return base + s * L::stage; };
-    auto a_tile = [&](int s) { return base + s * L::stage + L::w_tma; };
-    auto w_dq = [&](int d) { return base + STAGES * L::stage + d * L::dq_bytes; };
+    auto pfull_bar = [&](int p) { return smem_u32(bars + 2 * STAGES + p); };
+    auto pempty_bar = [&](int p) { return smem_u32(bars + 2 * STAGES + SP + p); };
+    auto dqf_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + 2 * SP + d); };
+    auto dqe_bar = [&](int d) { return smem_u32(bars + 2 * STAGES + 2 * SP + DQ + d); };
+    auto accf_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * SP + 2 * DQ + b); };
+    auto acce_bar = [&](int b) { return smem_u32(bars + 2 * STAGES + 2 * SP + 2 * DQ + 2 + b); };
+    const uint32_t final_bar = smem_u32(bars + 2 * STAGES + 2 * SP + 2 * DQ + 4);
+    // dense / int8: stage s = [weight slab | activation slab]; packed: stage s = activation slab
+    auto w_tma = [&](int s) { return base + s * (L::w_bytes + L::a_bytes); };
+    auto a_tile = [&](int s) {
+        return L::packed ? base + s * L::a_bytes : base + s * (L::w_bytes + L::a_bytes) + L::w_bytes;
+    };
+    auto pw_tile = [&](int p) { return base + L::pw_off + p * L::pw_bytes; };
+    auto w_dq = [&](int d) { return base + L::dq_off + d * L::dq_bytes; };
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
+        }
+        for (int p = 0; p < SP; ++p) {
+            mbar_init(pfull_bar(p), 1);
+            mbar_init(pempty_bar(p), 256);
         }
         for (int d = 0; d < DQ; ++d) {
             mbar_init(dqf_bar(d), 256);
@@ -296,9 +316,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 
     if (warp == 4) {
         if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            constexpr uint32_t kTx = L::w_tma + L::a_bytes;
-            const int wx_per_kb = T::packed ? 8 : T::k_per_slab;   // x units of tm_w per slab
+            // ---------------- TMA producer (weight + activation slabs, or activations) --------
+            constexpr uint32_t kTx = L::packed ? L::a_bytes : L::w_bytes + L::a_bytes;
             int it = 0;
             bool stop = false;
             for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
@@ -311,7 +330,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     }
                     mbar_expect_tx(full_bar(s), kTx);
                     const int kb = w.kb0 + i;
-                    tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * wx_per_kb, w.n0);
+                    if constexpr (!L::packed)
+                        tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * T::k_per_slab,
+                                    w.n0);
                     tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kb * T::k_per_slab, w.t0);
                 }
             }
@@ -319,6 +340,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             for (int i = max(0, it - STAGES); i < it; ++i) {
                 int dummy_abort = 0;
                 mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+            }
+        }
+    } else if (warp == 6) {
+        if (L::packed && lane == 0) {
+            // ---------------- TMA producer (packed weight slabs) ----------------
+            int it = 0;
+            bool stop = false;
+            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                for (int i = 0; i < w.nk; ++i, ++it) {
+                    const int p = it % SP;
+                    if (!mbar_wait(pempty_bar(p), ((it / SP) & 1) ^ 1, abort_flag, err)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_expect_tx(pfull_bar(p), L::pw_bytes);
+                    tma_load_2d(smem_u32(pw_tile(p)), &tm_w, pfull_bar(p), (w.kb0 + i) * 8, w.n0);
+                }
+            }
+            for (int i = max(0, it - SP); i < it; ++i) {
+                int dummy_abort = 0;
+                mbar_wait(pfull_bar(i % SP), (i / SP) & 1, &dummy_abort, nullptr);
             }
         }
     } else if (warp == 5) {
@@ -373,52 +416,154 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             const int dq = tid - 256;
             const int r = dq & 127, h = dq >> 7;
             const int G = K / gs;
-            int u = blockIdx.x, i = 0, it = 0;
-            Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
-            auto skip_empty = [&]() {
-                while (u < units && i >= w.nk) {
+            // cursor over this CTA's slabs: unit u (position i inside it, w its coordinates)
+            struct Cursor {
+                int u, i;
+                Unit w;
+            };
+            auto settle = [&](Cursor &c) {
+                while (c.u < units && c.i >= c.w.nk) {
+                    c.u += gridDim.x;
+                    c.i = 0;
+                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                }
+            };
+            Cursor cur{(int)blockIdx.x, 0, unit_of(blockIdx.x, n_tiles, t_tiles, BN, nkb, kb_per_split)};
+            settle(cur);
+            // Scales and zeros. Per slab a thread needs s[n][g] and z[n][g] of its row n. Loading
+            // those 2-byte values one slab at a time makes every warp touch 32 rows (32 sectors)
+            // per load, which saturates the LSU. Instead each thread keeps a window of 8
+            // consecutive groups of its row in registers (one 16-byte load for s, one for z) and
+            // prefetches the following window while it works through the current one. This needs
+            // G % 8 == 0 and 16-byte aligned scale / zero arrays; otherwise the values are
+            // loaded per slab, kLook slabs ahead.
+            const bool windowed = MODE == kW4A16 && G % 8 == 0 &&
+                                  (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
+                                  (reinterpret_cast<uintptr_t>(Z) & 15) == 0;
+            // group of a thread's half slab; a shift when the group size is a power of two
+            const int gs_shift = (gs & (gs - 1)) == 0 ? __ffs(gs) - 1 : -1;
+            auto group_of = [&](const Cursor &c) {
+                const int k = (c.w.kb0 + c.i) * 64 + 32 * h;
+                return min(gs_shift >= 0 ? k >> gs_shift : k / gs, G - 1);
+            };
+            struct Window {
+                int u, gb;                 // unit and first group (multiple of 8); u < 0: none
+                uint4 s, z;                // fp16 s and z of groups gb .. gb+7 of this row
+            };
+            auto load_window = [&](Window &wnd, int u, const Unit &w, int gb) {
+                wnd.u = u;
+                wnd.gb = gb;
+                if (u >= units) return;
+                const size_t off = (size_t)min(w.n0 + r, N - 1) * G + gb;
+                wnd.s = ld_cached_v4(S + off);
+                wnd.z = Z ? ld_cached_v4(Z + off) : make_uint4(0u, 0u, 0u, 0u);
+            };
+            // the window after wnd in this CTA's walk (same unit, or the next unit's first one)
+            auto next_window = [&](Window &out, const Window &wnd) {
+                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                const int g_last = min(((w.kb0 + w.nk) * 64 - 1) / gs, G - 1);
+                if (wnd.gb + 8 <= g_last) {
+                    load_window(out, wnd.u, w, wnd.gb + 8);
+                    return;
+                }
+                int u = wnd.u + gridDim.x;
+                Unit nw = w;
+                while (u < units) {
+                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                    if (nw.nk > 0) break;
                     u += gridDim.x;
-                    i = 0;
-                    if (u < units) w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
                 }
+                load_window(out, u, nw, (min((nw.kb0 * 64) / gs, G - 1)) & ~7);
             };
-            // (scale, -zero*scale) of slab i of unit w for this thread, as fp16 pairs
-            auto fetch = [&](const Unit &ww, int ii, float &sc, float &zz) {
-                const int n = min(ww.n0 + r, N - 1);
-                const int g = min(((ww.kb0 + ii) * 64 + 32 * h) / gs, G - 1);
-                sc = half_bits_to_float(ld_cached_u16(S + (size_t)n * G + g));
-                zz = Z ? half_bits_to_float(ld_cached_u16(Z + (size_t)n * G + g)) : 0.f;
-            };
-            skip_empty();
-            float sc = 0.f, zz = 0.f;
-            if (MODE == kW4A16 && u < units) fetch(w, i, sc, zz);
-            while (u < units) {
-                // position of the next slab, and its scale / zero in flight
-                int u2 = u, i2 = i + 1;
-                Unit w2 = w;
-                while (u2 < units && i2 >= w2.nk) {
-                    u2 += gridDim.x;
-                    i2 = 0;
-                    if (u2 < units) w2 = unit_of(u2, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            // the current window as fp16 pairs ready for the upcast: s and fp16(-z * s)
+            uint4 win_s = make_uint4(0u, 0u, 0u, 0u), win_nz = make_uint4(0u, 0u, 0u, 0u);
+            auto make_current = [&](const Window &wnd) {
+                const uint32_t sv[4] = {wnd.s.x, wnd.s.y, wnd.s.z, wnd.s.w};
+                const uint32_t zv[4] = {wnd.z.x, wnd.z.y, wnd.z.z, wnd.z.w};
+                uint32_t nz[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 sf = __half22float2(*reinterpret_cast<const __half2 *>(&sv[q]));
+                    const float2 zf = __half22float2(*reinterpret_cast<const __half2 *>(&zv[q]));
+                    nz[q] = pack_half2_rn(-zf.x * sf.x, -zf.y * sf.y);
                 }
-                float sc2 = 0.f, zz2 = 0.f;
-                if (MODE == kW4A16 && u2 < units) fetch(w2, i2, sc2, zz2);
-                const int s = it % STAGES, d = it % DQ;
+                win_s = wnd.s;
+                win_nz = make_uint4(nz[0], nz[1], nz[2], nz[3]);
+            };
+            // element j (0..7) of v, duplicated into both halves
+            auto pick2 = [](const uint4 &v, int j) {
+                const uint32_t lo = (j & 2) ? v.y : v.x, hi = (j & 2) ? v.w : v.z;
+                const uint32_t wv = (j & 4) ? hi : lo;
+                return prmt(wv, wv, (j & 1) ? 0x3232u : 0x1010u);
+            };
+            Window wcur{-1, 0, {}, {}}, wnxt{-1, 0, {}, {}};
+            if (windowed && cur.u < units) {
+                load_window(wcur, cur.u, cur.w, group_of(cur) & ~7);
+                make_current(wcur);
+                next_window(wnxt, wcur);
+            }
+            // per-slab fallback: scale and zero loaded kLook slabs ahead
+            constexpr int kLook = 4;
+            float sc[kLook], zz[kLook];
+            Cursor ahead = cur;
+            auto fetch = [&](const Cursor &c, float &s_out, float &z_out) {
+                if (MODE != kW4A16 || windowed || c.u >= units) {
+                    s_out = 0.f;
+                    z_out = 0.f;
+                    return;
+                }
+                const int n = min(c.w.n0 + r, N - 1);
+                const int g = group_of(c);
+                s_out = half_bits_to_float(ld_cached_u16(S + (size_t)n * G + g));
+                z_out = Z ? half_bits_to_float(ld_cached_u16(Z + (size_t)n * G + g)) : 0.f;
+            };
+#pragma unroll
+            for (int q = 0; q < kLook; ++q) {
+                fetch(ahead, sc[q], zz[q]);
+                ++ahead.i;
+                settle(ahead);
+            }
+            int it = 0;
+            while (cur.u < units) {
+                const int p = it % SP, d = it % DQ;
+                uint32_t sc2 = 0u, nz2 = 0u;             // (s, s) and (-z s, -z s) in fp16
+                if (windowed) {
+                    const int g = group_of(cur);
+                    if (wcur.u != cur.u || g < wcur.gb || g >= wcur.gb + 8) {
+                        if (wnxt.u == cur.u && g >= wnxt.gb && g < wnxt.gb + 8) wcur = wnxt;
+                        else load_window(wcur, cur.u, cur.w, g & ~7);
+                        make_current(wcur);
+                        next_window(wnxt, wcur);
+                    }
+                    sc2 = pick2(win_s, g - wcur.gb);
+                    nz2 = pick2(win_nz, g - wcur.gb);
+                } else if (MODE == kW4A16) {
+                    sc2 = half2_bcast(sc[0]);
+                    nz2 = half2_bcast(-zz[0] * sc[0]);
+#pragma unroll
+                    for (int q = 0; q + 1 < kLook; ++q) {   // shift the window (static indices)
+                        sc[q] = sc[q + 1];
+                        zz[q] = zz[q + 1];
+                    }
+                    fetch(ahead, sc[kLook - 1], zz[kLook - 1]);
+                    ++ahead.i;
+                    settle(ahead);
+                }
+                if (!mbar_wait(pfull_bar(p), (it / SP) & 1, abort_flag, err)) break;
+                const uint32_t *packed = reinterpret_cast<const uint32_t *>(pw_tile(p));
+                const uint4 pk = *reinterpret_cast<const uint4 *>(packed + r * 8 +
+                                                                 4 * (h ^ ((r >> 2) & 1)));
+                mbar_arrive(pempty_bar(p));          // the packed slot is free once read
                 if (!mbar_wait(dqe_bar(d), ((it / DQ) & 1) ^ 1, abort_flag, err)) break;
-                if (!mbar_wait(full_bar(s), (it / STAGES) & 1, abort_flag, err)) break;
-                const uint32_t *packed = reinterpret_cast<const uint32_t *>(w_tma(s));
                 if constexpr (MODE == kW4A16)
-                    dequant_w4(packed, w_dq(d), r, h, half2_bcast(sc), half2_bcast(-zz * sc));
+                    dequant_w4(pk, w_dq(d), r, h, sc2, nz2);
                 else
-                    dequant_w2(packed, w_dq(d), r, h);
+                    dequant_w2(pk, w_dq(d), r, h);
                 fence_proxy_async_smem();
                 mbar_arrive(dqf_bar(d));
                 ++it;
-                u = u2;
-                i = i2;
-                w = w2;
-                sc = sc2;
-                zz = zz2;
+                ++cur.i;
+                settle(cur);
             }
         }
     } else if (warp < 4) {
@@ -622,6 +767,12 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
     if (p.op == QG_OP_W8A8 && p.K % 16) return false;
     if (p.op == QG_OP_DENSE_F16 && p.K % 8) return false;
     return true;
+}
+
+int tc_dq_buffers(int op, int bn, int stages)
+{
+    const int mode = mode_of(op);
+    return dq_buffers(mode == kW4A16 || mode == kW2A8, bn, stages);
 }
 
 int tc_max_stages(int op, int bn)

@@ -38,6 +38,7 @@
 #ifndef QGEMM_H_
 #define QGEMM_H_
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -95,6 +96,28 @@ typedef struct qgemm_config_t {
 qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, const void *zeros,
                       void *C, int M, int N, int K, int group_size, int split_k, int has_zero,
                       cudaStream_t stream);
+
+/*
+ * W4A16 with deterministic split-K: the fp32-workspace form of parallel-k (hidet-org/hidet issue
+ * #364, parallel-k discussion; qgemm_w4a16 with split_k > 1 is the atomic form). Operands and
+ * result as qgemm_w4a16. Each of the split_k (>= 1, given explicitly) parts of the K reduction
+ * writes its fp32 partial tile into `workspace`; the last part to finish a tile adds all partial
+ * tiles in part order and rounds once to fp16. The result is bit-identical from run to run and
+ * carries no fp16 rounding of partial sums.
+ * Runs on the small-M streaming kernel: requires group_size % 128 == 0 (or -1 / 0 with
+ * K % 128 == 0); any M is accepted, M <= 16 is what it is built for.
+ * workspace: caller-owned device memory, 256-byte aligned, at least
+ * qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k) bytes. Its contents on entry do not
+ * matter (the call clears the part that must start at zero). Calls that share a workspace must
+ * not overlap on the GPU.
+ */
+qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *scales,
+                                 const void *zeros, void *C, int M, int N, int K, int group_size,
+                                 int split_k, int has_zero, void *workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes qgemm_w4a16_splitk_f32 needs for these arguments (0 if they are invalid). */
+size_t qgemm_w4a16_workspace_bytes(int M, int N, int K, int group_size, int split_k);
 
 /*
  * W8A8. A: int8 [M, K]. W: int8 [N, K]. C: int32 [M, N] = sum_k A[m,k] * W[n,k], exact

@@ -38,7 +38,8 @@ class Oracle:
         L = ctypes.CDLL(path)
         L.orc_half_to_double.restype = ctypes.c_double
         L.orc_half_to_double.argtypes = [ctypes.c_uint16]
-        for name in ("orc_pack_int4", "orc_unpack_int4", "orc_pack_int2", "orc_unpack_int2"):
+        for name in ("orc_pack_int4", "orc_unpack_int4", "orc_pack_int2", "orc_unpack_int2",
+                     "orc_pack_int4_interleaved", "orc_unpack_int4_interleaved"):
             getattr(L, name).argtypes = [_ptr, _ptr, _i64, _i64]
             getattr(L, name).restype = ctypes.c_int
         L.orc_decode_half.argtypes = [_ptr, _ptr, _i64]
@@ -86,6 +87,21 @@ class Oracle:
         N = packed.shape[0]
         out = np.empty((N, K), dtype=np.uint8)
         _check(self.L.orc_unpack_int4(_p(packed), _p(out), N, K), "unpack_int4")
+        return out
+
+    def pack_int4_interleaved(self, codes: np.ndarray) -> np.ndarray:
+        codes = np.ascontiguousarray(codes, dtype=np.uint8)
+        N, K = codes.shape
+        out = np.empty((N, K // 8), dtype=np.uint32)
+        _check(self.L.orc_pack_int4_interleaved(_p(codes), _p(out), N, K), "pack_int4_interleaved")
+        return out
+
+    def unpack_int4_interleaved(self, packed: np.ndarray, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        N = packed.shape[0]
+        out = np.empty((N, K), dtype=np.uint8)
+        _check(self.L.orc_unpack_int4_interleaved(_p(packed), _p(out), N, K),
+               "unpack_int4_interleaved")
         return out
 
     def pack_int2(self, vals: np.ndarray) -> np.ndarray:
@@ -221,6 +237,8 @@ def max_threads() -> int: return get().max_threads()
 def half_to_double(b): return get().half_to_double(b)
 def pack_int4(c): return get().pack_int4(c)
 def unpack_int4(p, K): return get().unpack_int4(p, K)
+def pack_int4_interleaved(c): return get().pack_int4_interleaved(c)
+def unpack_int4_interleaved(p, K): return get().unpack_int4_interleaved(p, K)
 def pack_int2(v): return get().pack_int2(v)
 def unpack_int2(p, K): return get().unpack_int2(p, K)
 def w4a16(*a, **k): return get().w4a16(*a, **k)

@@ -91,6 +91,36 @@ int orc_unpack_int4(const uint32_t *packed, uint8_t *codes, int64_t N, int64_t K
     return ORC_OK;
 }
 
+/*
+ * Interleaved int4 packing (the pre-shuffled layout): inside each word, code k = 8j + e sits in
+ * nibble ILV_POS[e] = (e % 2) * 4 + e / 2, i.e. nibbles 0..7 hold codes 0, 2, 4, 6, 1, 3, 5, 7 of
+ * the word. Reading nibbles i and i + 4 of a word then gives two codes adjacent in k.
+ */
+static const int ILV_POS[8] = {0, 4, 1, 5, 2, 6, 3, 7};
+
+int orc_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 8) return ORC_BAD_ARGS;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 8; ++j) {
+            uint32_t word = 0;
+            for (int e = 0; e < 8; ++e)
+                word |= (uint32_t)(codes[n * K + 8 * j + e] & 0xF) << (4 * ILV_POS[e]);
+            packed[n * (K / 8) + j] = word;
+        }
+    return ORC_OK;
+}
+
+int orc_unpack_int4_interleaved(const uint32_t *packed, uint8_t *codes, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 8) return ORC_BAD_ARGS;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            codes[n * K + k] =
+                (uint8_t)((packed[n * (K / 8) + k / 8] >> (4 * ILV_POS[k % 8])) & 0xF);
+    return ORC_OK;
+}
+
 /* packed[n, j] = sum_i (vals[n, 16j+i] & 3) << 2i   (two's-complement 2-bit fields) */
 int orc_pack_int2(const int8_t *vals, uint32_t *packed, int64_t N, int64_t K)
 {

@@ -175,12 +175,35 @@ def test_tc_split_fills_the_gpu():
 
 def test_tc_config_limits():
     M, N, K = 256, 512, 1024
-    # packed weights: 5 TMA stages of 36 KB plus two 16 KB dequant buffers fit (213 KB)
-    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 5))
-    for bad in (_tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
+    # packed weights at a 256-token tile: 4 activation stages (128 KB) + 12 packed slabs (48 KB)
+    # + 3 upcast buffers (48 KB) fit; a fifth activation stage does not
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 4))
+    for bad in (_tc(256, 5), _tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
         with pytest.raises(qg.QGemmError):
             qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, bad)
     qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 4))
     with pytest.raises(qg.QGemmError):
         qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 5))
     qg.qgemm_clear_configs()
+
+
+def test_workspace_bytes():
+    # counters (one per 16-row x 8-token tile, 256-byte aligned) + split_k planes of M x N fp32
+    assert qg.qgemm_w4a16_workspace_bytes(1, 4096, 4096, 128, 4) == 1024 + 4 * 4096 * 4
+    assert qg.qgemm_w4a16_workspace_bytes(16, 100, 1024, 128, 3) == 256 + 3 * 16 * 100 * 4
+    assert qg.qgemm_w4a16_workspace_bytes(1, 4096, 4096, 128, 0) == 0
+    assert qg.qgemm_w4a16_workspace_bytes(1, 4096, 4000, 128, 2) == 0
+
+
+def test_splitk_f32_validation_without_gpu():
+    L = qg.lib()
+    ws = ctypes.c_void_p(0x100000)
+    need = qg.qgemm_w4a16_workspace_bytes(1, 64, 256, 128, 2)
+    assert L.qgemm_w4a16_splitk_f32(A, W, S, Z, C, 1, 64, 256, 128, 0, 1, ws, need, None) == \
+        qg.QG_ERR_INVALID_ARG                                         # split_k must be given
+    assert L.qgemm_w4a16_splitk_f32(A, W, S, Z, C, 1, 64, 256, 64, 2, 1, ws, need, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE                                   # group size 64
+    assert L.qgemm_w4a16_splitk_f32(A, W, S, Z, C, 1, 64, 256, 128, 2, 1, ws, need - 4, None) == \
+        qg.QG_ERR_INVALID_ARG                                         # workspace too small
+    assert L.qgemm_w4a16_splitk_f32(A, W, S, Z, C, 1, 64, 256, 128, 2, 1,
+                                    ctypes.c_void_p(0x100010), need, None) == qg.QG_ERR_ALIGNMENT

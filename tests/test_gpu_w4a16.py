@@ -192,3 +192,40 @@ def test_w4a16_tma_kernel_long_k(stages, split_k):
         assert_fp16_close(case.run(), case.ref_full(), f"stages={stages} split={split_k}")
     finally:
         qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, None)
+
+
+# ---- deterministic split-K through an fp32 workspace ------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (5, 200, 1024), (16, 130, 2048), (9, 64, 4096)])
+@pytest.mark.parametrize("split_k", [1, 2, 3, 8])
+def test_w4a16_splitk_f32_parity_and_determinism(M, N, K, split_k):
+    case = W4Case(M, N, K, 128, 1, seed=M + split_k)
+    need = qg.qgemm_w4a16_workspace_bytes(M, N, K, 128, split_k)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)      # contents must not matter
+    a = qg.qgemm_w4a16_splitk_f32(case.A, case.Wq, case.S, case.Z, group_size=128,
+                                  split_k=split_k, workspace=ws).clone()
+    b = qg.qgemm_w4a16_splitk_f32(case.A, case.Wq, case.S, case.Z, group_size=128,
+                                  split_k=split_k, workspace=ws).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)                     # part order is fixed: bit-identical reruns
+    assert_fp16_close(a, case.ref_full(), f"splitk_f32 split={split_k}")
+
+
+def test_w4a16_splitk_f32_no_zero_point_and_per_channel():
+    case = W4Case(3, 256, 2048, -1, 0, seed=5)
+    C = qg.qgemm_w4a16_splitk_f32(case.A, case.Wq, case.S, None, group_size=-1, split_k=4)
+    assert_fp16_close(C, case.ref_full(), "per-channel, no zero")
+
+
+def test_w4a16_splitk_f32_rejects_bad_workspace():
+    case = W4Case(2, 128, 1024, 128, 1)
+    need = qg.qgemm_w4a16_workspace_bytes(2, 128, 1024, 128, 4)
+    small = torch.empty(need - 256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_w4a16_splitk_f32(case.A, case.Wq, case.S, case.Z, split_k=4, workspace=small)
+    big = torch.empty(need + 512, dtype=torch.uint8, device=DEV)
+    with pytest.raises(qg.QGemmError):                   # 16-byte offset breaks 256-byte alignment
+        qg.qgemm_w4a16_splitk_f32(case.A, case.Wq, case.S, case.Z, split_k=4, workspace=big[16:])
+    with pytest.raises(qg.QGemmError):                   # group size 64: not this kernel's
+        c64 = W4Case(2, 128, 1024, 64, 1)
+        qg.qgemm_w4a16_splitk_f32(c64.A, c64.Wq, c64.S, c64.Z, group_size=64, split_k=2)

@@ -67,6 +67,25 @@ def test_pack_golden_words():
     check_pack_fixtures(oracle.get())
 
 
+def check_pack_interleaved(orc):
+    for codes, word in _fixture_rows("pack_int4_interleaved.txt"):
+        got = orc.pack_int4_interleaved(np.array([codes], dtype=np.uint8))
+        assert int(got[0, 0]) == word, (codes, hex(int(got[0, 0])))
+        assert orc.unpack_int4_interleaved(np.array([[word]], dtype=np.uint32), 8).tolist() == [codes]
+    # the same codes in both layouts: a fixed permutation of the nibbles of every word
+    codes = synth.uniform_int((7, 64), 0, 15, 8, synth.TID_W, np.uint8)
+    nat = orc.pack_int4(codes)
+    ilv = orc.pack_int4_interleaved(codes)
+    assert np.array_equal(orc.unpack_int4_interleaved(ilv, 64), codes)
+    perm = [0, 2, 4, 6, 1, 3, 5, 7]           # nibble i of the interleaved word = code perm[i]
+    for i, e in enumerate(perm):
+        assert np.array_equal((ilv >> (4 * i)) & 0xF, (nat >> (4 * e)) & 0xF)
+
+
+def test_pack_interleaved():
+    check_pack_interleaved(oracle.get())
+
+
 def test_pack_roundtrip_random():
     codes = synth.uniform_int((37, 256), 0, 15, 3, synth.TID_W, np.uint8)
     assert np.array_equal(oracle.unpack_int4(oracle.pack_int4(codes), 256), codes)
@@ -322,11 +341,14 @@ MUTANTS = [
     ("pack order reversed", "<< (4 * i);", "<< (4 * (7 - i));"),
     ("pack code not masked", "(uint32_t)(codes[n * K + 8 * j + i] & 0xF)",
      "(uint32_t)(codes[n * K + 8 * j + i])"),
+    ("interleaved layout wrong", "static const int ILV_POS[8] = {0, 4, 1, 5, 2, 6, 3, 7};",
+     "static const int ILV_POS[8] = {0, 1, 2, 3, 4, 5, 6, 7};"),
+    ("interleaved unpack shift", "(4 * ILV_POS[k % 8])) & 0xF)", "(4 * (k % 8))) & 0xF)"),
     ("int2 pack not masked", "((uint8_t)vals[n * K + 16 * j + i] & 3u)",
      "((uint8_t)vals[n * K + 16 * j + i])"),
 ]
 
-PINS = [check_half_decoder, check_pack_fixtures, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
+PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
         check_w4_one_hot_reads_single_weight, check_w4_constant_closed_form,
         check_w4_per_channel_equals_one_group, check_w4_parallel_k_additivity,
         check_w4_elementwise_matches_full, check_dense_is_numpy_matmul,
