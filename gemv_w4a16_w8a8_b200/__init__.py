@@ -27,12 +27,12 @@ QG_ERR_DEVICE_TIMEOUT = 5
 QG_ERR_NOT_SM100 = 6
 QG_ERR_BAD_CONFIG = 7
 
-OP_W4A16, OP_W8A8, OP_W2A8, OP_DENSE_F16 = 0, 1, 2, 3
+OP_W4A16, OP_W8A8, OP_W2A8, OP_DENSE_F16, OP_W4A16_INTERLEAVED = 0, 1, 2, 3, 4
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 
 # every symbol include/qgemm.h declares
 EXPORTS = (
-    "qgemm_w4a16", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
     "qgemm_version",
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, i32 = ctypes.c_void_p, ctypes.c_int
         L.qgemm_w4a16.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.qgemm_w4a16_interleaved.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.quant_pack_int4_interleaved.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_w4a16_splitk_f32.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
                                              ctypes.c_size_t, vp]
         L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
@@ -159,6 +161,42 @@ def qgemm_w4a16(A, Wq, scales, zeros=None, C=None, group_size: int = 128, split_
                            group_size, split_k, int(zeros is not None), _stream(stream))
     _check(st, "qgemm_w4a16")
     return C
+
+
+def qgemm_w4a16_interleaved(A, Wq, scales, zeros=None, C=None, group_size: int = 128,
+                            split_k: int = 0, stream=None):
+    """As qgemm_w4a16, with Wq from quant_pack_int4_interleaved."""
+    torch = _torch()
+    _need(A, torch.float16, 2, "A")
+    _need(Wq, (torch.int32, torch.uint32), 2, "Wq")
+    _need(scales, torch.float16, 2, "scales")
+    if zeros is not None:
+        _need(zeros, torch.float16, 2, "zeros")
+    M, K = A.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] * 8 != K:
+        raise ValueError(f"Wq must be [N, K/8] = [{N}, {K // 8}], got {tuple(Wq.shape)}")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _need(C, torch.float16, 2, "C")
+    st = lib().qgemm_w4a16_interleaved(_ptr(A), _ptr(Wq), _ptr(scales), _ptr(zeros), _ptr(C), M,
+                                       N, K, group_size, split_k, int(zeros is not None),
+                                       _stream(stream))
+    _check(st, "qgemm_w4a16_interleaved")
+    return C
+
+
+def quant_pack_int4_interleaved(codes, out=None, stream=None):
+    """codes uint8 [N,K] -> int32 [N,K/8] in the interleaved layout (nibbles 0..7 of each word
+    hold codes 0,2,4,6,1,3,5,7 of its eight)."""
+    torch = _torch()
+    _need(codes, torch.uint8, 2, "codes")
+    N, K = codes.shape
+    if out is None:
+        out = torch.empty((N, K // 8), dtype=torch.int32, device=codes.device)
+    _check(lib().quant_pack_int4_interleaved(_ptr(codes), _ptr(out), 0, N, K, -1, 1, 0,
+                                             _stream(stream)), "quant_pack_int4_interleaved")
+    return out
 
 
 def qgemm_w4a16_workspace_bytes(M: int, N: int, K: int, group_size: int, split_k: int) -> int:

@@ -84,7 +84,7 @@ int sm_count_or_default()
 
 int effective_gs(int op, int K, int group_size)
 {
-    if (op != QG_OP_W4A16) return K;
+    if (op != QG_OP_W4A16 && op != QG_OP_W4A16_INTERLEAVED) return K;
     return group_size <= 0 ? K : group_size;
 }
 
@@ -93,12 +93,13 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Shape / flag rules shared by the matmul entry points, the planner and the tuner.
 qg_status check_shape(int op, int M, int N, int K, int group_size, int has_zero, int split_k)
 {
-    if (op < QG_OP_W4A16 || op > QG_OP_DENSE_F16) return QG_ERR_INVALID_ARG;
+    if (op < QG_OP_W4A16 || op > QG_OP_W4A16_INTERLEAVED) return QG_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
     if (split_k > kMaxSplit) return QG_ERR_INVALID_ARG;
     if (has_zero != 0 && has_zero != 1) return QG_ERR_INVALID_ARG;
     switch (op) {
-    case QG_OP_W4A16: {
+    case QG_OP_W4A16:
+    case QG_OP_W4A16_INTERLEAVED: {
         if (K % 32) return QG_ERR_UNSUPPORTED_SHAPE;
         if (group_size < -1) return QG_ERR_INVALID_ARG;
         const int gs = effective_gs(op, K, group_size);
@@ -124,7 +125,8 @@ Problem make_problem(int op, const void *A, const void *W, const void *scales,
                      int has_zero)
 {
     Problem p;
-    p.op = op;
+    p.op = op == QG_OP_W4A16_INTERLEAVED ? QG_OP_W4A16 : op;
+    p.interleaved = op == QG_OP_W4A16_INTERLEAVED ? 1 : 0;
     p.A = A;
     p.W = W;
     p.scales = scales;
@@ -288,7 +290,8 @@ void ensure_cache_loaded_locked()
 
 Key key_of(const Problem &p)
 {
-    return Key(p.op, p.M, p.N, p.K, p.gs, p.has_zero);
+    return Key(p.interleaved ? (int)QG_OP_W4A16_INTERLEAVED : p.op, p.M, p.N, p.K, p.gs,
+               p.has_zero);
 }
 
 qgemm_config_t choose(const Problem &p, int split_k, int sms)
@@ -346,7 +349,7 @@ qg_status matmul(int op, const void *A, const void *W, const void *scales, const
     qg_status s = check_shape(op, M, N, K, group_size, has_zero, split_k);
     if (s != QG_OK) return s;
     if (!A || !W || !C) return QG_ERR_INVALID_ARG;
-    if (op == QG_OP_W4A16) {
+    if (op == QG_OP_W4A16 || op == QG_OP_W4A16_INTERLEAVED) {
         if (!scales) return QG_ERR_INVALID_ARG;
         if ((zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
         if (!aligned(scales, 2) || (zeros && !aligned(zeros, 2))) return QG_ERR_ALIGNMENT;
@@ -475,6 +478,32 @@ qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *
     return QG_OK;
 }
 
+qg_status qgemm_w4a16_interleaved(const void *A, const uint32_t *Wq, const void *scales,
+                                  const void *zeros, void *C, int M, int N, int K, int group_size,
+                                  int split_k, int has_zero, cudaStream_t stream)
+{
+    return matmul(QG_OP_W4A16_INTERLEAVED, A, Wq, scales, zeros, C, M, N, K, group_size, split_k,
+                  has_zero, stream);
+}
+
+qg_status quant_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int M, int N, int K,
+                                      int group_size, int split_k, int has_zero,
+                                      cudaStream_t stream)
+{
+    (void)M; (void)group_size; (void)split_k; (void)has_zero;
+    if (!codes || !packed || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+    if (K % 32) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(codes, 16) || !aligned(packed, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_pack_int4_interleaved(codes, packed, N, K, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N, int K,
                      int group_size, int split_k, int has_zero, cudaStream_t stream)
 {
@@ -565,8 +594,9 @@ qg_status qgemm_tune(int op, const void *A, const void *W, const void *scales,
 {
     qg_status s = check_shape(op, M, N, K, group_size, has_zero, 0);
     if (s != QG_OK) return s;
-    if (!A || !W || !C || (op == QG_OP_W4A16 && !scales)) return QG_ERR_INVALID_ARG;
-    if (op == QG_OP_W4A16 && (zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+    const bool w4 = op == QG_OP_W4A16 || op == QG_OP_W4A16_INTERLEAVED;
+    if (!A || !W || !C || (w4 && !scales)) return QG_ERR_INVALID_ARG;
+    if (w4 && (zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
     if (!aligned(A, 16) || !aligned(W, 16) || !aligned(C, 16)) return QG_ERR_ALIGNMENT;
     DeviceInfo *d = nullptr;
     s = probe_device(&d);

@@ -41,7 +41,8 @@ __device__ __forceinline__ void load_words(uint32_t (&w)[WPT], const uint32_t *p
     }
 }
 
-// Exact fp16 pairs of the eight codes of one word: (q0,q4) (q1,q5) (q2,q6) (q3,q7).
+// Exact fp16 pairs of the eight codes of one word: (q0,q4) (q1,q5) (q2,q6) (q3,q7) for the
+// natural packing, (q0,q1) (q2,q3) (q4,q5) (q6,q7) for the interleaved one.
 __device__ __forceinline__ void upcast_word(uint32_t w, uint32_t (&h)[4])
 {
     constexpr uint32_t kMagic = 0x64006400u;  // fp16 1024.0 | 1024.0
@@ -273,24 +274,25 @@ gemv_w4a16_kernel(const __half *__restrict__ A, const uint32_t *__restrict__ Wq,
 }
 
 template <int WPT, int RB, int NT, bool ILV>
-void launch_ilv(const Problem &p, int split_k, cudaStream_t stream);
+void launch_ilv(const Problem &p, int split_k, cudaStream_t stream)
+{
+    constexpr int KB = 32 * WPT;
+    const int nkb = p.K / KB;
+    const int kbps = (nkb + split_k - 1) / split_k;
+    const int splits = (nkb + kbps - 1) / kbps;   // drop trailing empty splits
+    dim3 grid((p.N + 16 * RB - 1) / (16 * RB), splits, (p.M + 8 * NT - 1) / (8 * NT));
+    gemv_w4a16_kernel<WPT, RB, NT, ILV><<<grid, kWarps * 32, 0, stream>>>(
+        static_cast<const __half *>(p.A), static_cast<const uint32_t *>(p.W),
+        static_cast<const __half *>(p.scales),
+        p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, static_cast<__half *>(p.C),
+        p.M, p.N, p.K, p.gs, kbps, split_k > 1 ? 1 : 0);
+}
 
 template <int WPT, int RB, int NT>
 void launch_one(const Problem &p, int split_k, cudaStream_t stream)
 {
     if (p.interleaved) launch_ilv<WPT, RB, NT, true>(p, split_k, stream);
     else launch_ilv<WPT, RB, NT, false>(p, split_k, stream);
-}
-    constexpr int KB = 32 * WPT;
-    const int nkb = p.K / KB;
-    const int kbps = (nkb + split_k - 1) / split_k;
-    const int splits = (nkb + kbps - 1) / kbps;   // drop trailing empty splits
-    dim3 grid((p.N + 16 * RB - 1) / (16 * RB), splits, (p.M + 8 * NT - 1) / (8 * NT));
-    gemv_w4a16_kernel<WPT, RB, NT><<<grid, kWarps * 32, 0, stream>>>(
-        static_cast<const __half *>(p.A), static_cast<const uint32_t *>(p.W),
-        static_cast<const __half *>(p.scales),
-        p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, static_cast<__half *>(p.C),
-        p.M, p.N, p.K, p.gs, kbps, split_k > 1 ? 1 : 0);
 }
 
 template <int WPT, int NT>

@@ -25,13 +25,24 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kKB = 128;                 // K values per k-block (16 packed words per row)
 
+// Activations paired like the codes the LOP3 upcast yields (natural packing: (a0,a4) (a1,a5)
+// (a2,a6) (a3,a7); interleaved packing: (a0,a1) (a2,a3) (a4,a5) (a6,a7)), and the pairs that
+// meet 16 q scaled by 1/16.
+template <bool ILV>
 __device__ __forceinline__ void act_pairs_scaled(const uint4 &v, uint32_t (&b)[4])
 {
     constexpr uint32_t kInv16 = 0x2C002C00u;   // fp16 1/16 in both halves
-    b[0] = prmt(v.x, v.z, 0x5410);                      // (a0, a4)
-    b[1] = hmul2_u32(prmt(v.x, v.z, 0x7632), kInv16);   // (a1, a5) / 16
-    b[2] = prmt(v.y, v.w, 0x5410);                      // (a2, a6)
-    b[3] = hmul2_u32(prmt(v.y, v.w, 0x7632), kInv16);   // (a3, a7) / 16
+    if constexpr (ILV) {
+        b[0] = v.x;
+        b[1] = hmul2_u32(v.y, kInv16);
+        b[2] = v.z;
+        b[3] = hmul2_u32(v.w, kInv16);
+    } else {
+        b[0] = prmt(v.x, v.z, 0x5410);
+        b[1] = hmul2_u32(prmt(v.x, v.z, 0x7632), kInv16);
+        b[2] = prmt(v.y, v.w, 0x5410);
+        b[3] = hmul2_u32(prmt(v.y, v.w, 0x7632), kInv16);
+    }
 }
 
 template <int RB, int NT, int STAGES> struct Layout {
@@ -45,7 +56,7 @@ template <int RB, int NT, int STAGES> struct Layout {
 };
 
 // RB: 16-row blocks per CTA (all four warps share them and split K).  NT: 8-token tiles.
-template <int RB, int NT, int STAGES>
+template <int RB, int NT, int STAGES, bool ILV>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__restrict__ A,
                       const __half *__restrict__ S, const __half *__restrict__ Z,
@@ -151,7 +162,7 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
 #pragma unroll
         for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) act_pairs_scaled(av[t][j], b[t][j]);
+            for (int j = 0; j < 4; ++j) act_pairs_scaled<ILV>(av[t][j], b[t][j]);
         float sc[RB][2], zr[RB][2];
 #pragma unroll
         for (int r = 0; r < RB; ++r)
@@ -307,12 +318,12 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
     }
 }
 
-template <int RB, int NT, int STAGES>
-cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
+template <int RB, int NT, int STAGES, bool ILV>
+cudaError_t launch_ilv(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
                        float *ws_part, unsigned int *ws_count)
 {
     using L = Layout<RB, NT, STAGES>;
-    auto kern = gemv_w4a16_tma_kernel<RB, NT, STAGES>;
+    auto kern = gemv_w4a16_tma_kernel<RB, NT, STAGES, ILV>;
     static std::mutex mu;
     static bool opted_in[64] = {};
     int dev = 0;
@@ -339,6 +350,15 @@ cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStr
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, static_cast<__half *>(p.C),
         p.M, p.N, p.K, p.gs, kbps, (split_k > 1 && !ws_part) ? 1 : 0, err, ws_part, ws_count);
     return cudaGetLastError();
+}
+
+template <int RB, int NT, int STAGES>
+cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
+                       float *ws_part, unsigned int *ws_count)
+{
+    return p.interleaved ? launch_ilv<RB, NT, STAGES, true>(p, split_k, err, stream, ws_part, ws_count)
+                         : launch_ilv<RB, NT, STAGES, false>(p, split_k, err, stream, ws_part,
+                                                             ws_count);
 }
 
 template <int RB, int NT>

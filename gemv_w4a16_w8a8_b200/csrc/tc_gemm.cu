@@ -30,7 +30,9 @@
 namespace qg {
 namespace {
 
-enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3 };
+enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3, kW4A16I = 4 };   // I: interleaved int4
+
+constexpr bool is_w4(int m) { return m == kW4A16 || m == kW4A16I; }
 
 constexpr int kThreads = 512;
 constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
@@ -53,7 +55,7 @@ template <int MODE>
 __device__ __forceinline__ void mma_issue(uint32_t dtm, uint64_t a, uint64_t b, uint32_t idesc,
                                           uint32_t accumulate)
 {
-    if constexpr (MODE == kDense || MODE == kW4A16) {
+    if constexpr (MODE == kDense || is_w4(MODE)) {
         asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtm),
                      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
@@ -94,11 +96,11 @@ __host__ __device__ constexpr uint32_t instr_desc()
 }
 
 template <int MODE> struct Traits {
-    static constexpr bool packed = (MODE == kW4A16 || MODE == kW2A8);
+    static constexpr bool packed = (is_w4(MODE) || MODE == kW2A8);
     static constexpr int w_tma_bytes = packed ? kRowsW * 32 : kRowsW * kSlabBytes;
     static constexpr int w_mma_bytes = packed ? kRowsW * kSlabBytes : 0;   // dequant target
-    static constexpr int k_per_slab = (MODE == kDense || MODE == kW4A16) ? 64 : 128;
-    static constexpr int c_bytes = (MODE == kDense || MODE == kW4A16) ? 2 : 4;
+    static constexpr int k_per_slab = (MODE == kDense || is_w4(MODE)) ? 64 : 128;
+    static constexpr int c_bytes = (MODE == kDense || is_w4(MODE)) ? 2 : 4;
 };
 
 // Shared memory.
@@ -147,6 +149,7 @@ template <int BN> constexpr uint32_t tmem_cols() { return 2 * BN < 32 ? 32u : (u
 // Upcast half a slab of packed int4 (p = words 4h..4h+3 of weight row r: 32 values of K, one
 // quantisation group) into fp16 (q - z) * s = fma(q, s, fp16(-z * s)), written in the
 // SWIZZLE_128B K-major layout the MMA reads.
+template <bool ILV>
 __device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, int h,
                                            uint32_t sc, uint32_t nz)
 {
@@ -157,15 +160,23 @@ __device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t w = words[j], w8 = w >> 8;
-        const uint32_t h0 = hsub2_u32(lop3_and_or(w, kLo, kMagic), kMagic);        // q0 q4
-        const uint32_t h1 = hfma2_u32(lop3_and_or(w, kHi, kMagic), kInv16, kNeg64); // q1 q5
-        const uint32_t h2 = hsub2_u32(lop3_and_or(w8, kLo, kMagic), kMagic);       // q2 q6
-        const uint32_t h3 = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);// q3 q7
+        // natural packing: (q0,q4) (q1,q5) (q2,q6) (q3,q7); interleaved: (q0,q1) .. (q6,q7)
+        const uint32_t h0 = hsub2_u32(lop3_and_or(w, kLo, kMagic), kMagic);
+        const uint32_t h1 = hfma2_u32(lop3_and_or(w, kHi, kMagic), kInv16, kNeg64);
+        const uint32_t h2 = hsub2_u32(lop3_and_or(w8, kLo, kMagic), kMagic);
+        const uint32_t h3 = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);
         uint4 o;
-        o.x = hfma2_u32(prmt(h0, h1, 0x5410), sc, nz);   // (q0, q1)
-        o.y = hfma2_u32(prmt(h2, h3, 0x5410), sc, nz);   // (q2, q3)
-        o.z = hfma2_u32(prmt(h0, h1, 0x7632), sc, nz);   // (q4, q5)
-        o.w = hfma2_u32(prmt(h2, h3, 0x7632), sc, nz);   // (q6, q7)
+        if constexpr (ILV) {
+            o.x = hfma2_u32(h0, sc, nz);
+            o.y = hfma2_u32(h1, sc, nz);
+            o.z = hfma2_u32(h2, sc, nz);
+            o.w = hfma2_u32(h3, sc, nz);
+        } else {
+            o.x = hfma2_u32(prmt(h0, h1, 0x5410), sc, nz);   // (q0, q1)
+            o.y = hfma2_u32(prmt(h2, h3, 0x5410), sc, nz);   // (q2, q3)
+            o.z = hfma2_u32(prmt(h0, h1, 0x7632), sc, nz);   // (q4, q5)
+            o.w = hfma2_u32(prmt(h2, h3, 0x7632), sc, nz);   // (q6, q7)
+        }
         *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }
 }
@@ -437,7 +448,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             // prefetches the following window while it works through the current one. This needs
             // G % 8 == 0 and 16-byte aligned scale / zero arrays; otherwise the values are
             // loaded per slab, kLook slabs ahead.
-            const bool windowed = MODE == kW4A16 && G % 8 == 0 &&
+            const bool windowed = is_w4(MODE) && G % 8 == 0 &&
                                   (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
                                   (reinterpret_cast<uintptr_t>(Z) & 15) == 0;
             // group of a thread's half slab; a shift when the group size is a power of two
@@ -507,7 +518,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             float sc[kLook], zz[kLook];
             Cursor ahead = cur;
             auto fetch = [&](const Cursor &c, float &s_out, float &z_out) {
-                if (MODE != kW4A16 || windowed || c.u >= units) {
+                if (!is_w4(MODE) || windowed || c.u >= units) {
                     s_out = 0.f;
                     z_out = 0.f;
                     return;
@@ -537,7 +548,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     }
                     sc2 = pick2(win_s, g - wcur.gb);
                     nz2 = pick2(win_nz, g - wcur.gb);
-                } else if (MODE == kW4A16) {
+                } else if (is_w4(MODE)) {
                     sc2 = half2_bcast(sc[0]);
                     nz2 = half2_bcast(-zz[0] * sc[0]);
 #pragma unroll
@@ -555,8 +566,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                                                                  4 * (h ^ ((r >> 2) & 1)));
                 mbar_arrive(pempty_bar(p));          // the packed slot is free once read
                 if (!mbar_wait(dqe_bar(d), ((it / DQ) & 1) ^ 1, abort_flag, err)) break;
-                if constexpr (MODE == kW4A16)
-                    dequant_w4(pk, w_dq(d), r, h, sc2, nz2);
+                if constexpr (is_w4(MODE))
+                    dequant_w4<MODE == kW4A16I>(pk, w_dq(d), r, h, sc2, nz2);
                 else
                     dequant_w2(pk, w_dq(d), r, h);
                 fence_proxy_async_smem();
@@ -646,7 +657,7 @@ int mode_of(int op)
 
 int smem_bytes(int mode, int bn, int stages)
 {
-    const bool packed = (mode == kW4A16 || mode == kW2A8);
+    const bool packed = (is_w4(mode) || mode == kW2A8);
     return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages));
 }
 
@@ -684,7 +695,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                       kRowsW, CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
                       CU_TENSOR_MAP_SWIZZLE_128B);
-    } else if constexpr (MODE == kW4A16) {
+    } else if constexpr (is_w4(MODE)) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
                       8, kRowsW, CU_TENSOR_MAP_SWIZZLE_32B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
@@ -772,7 +783,7 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
 int tc_dq_buffers(int op, int bn, int stages)
 {
     const int mode = mode_of(op);
-    return dq_buffers(mode == kW4A16 || mode == kW2A8, bn, stages);
+    return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages);
 }
 
 int tc_max_stages(int op, int bn)
@@ -788,7 +799,9 @@ cudaError_t launch_tc(const Problem &p, const qgemm_config_t &c, unsigned int *e
     switch (mode_of(p.op)) {
     case kDense: return launch_bn<kDense>(p, c, err, stream);
     case kW8A8: return launch_bn<kW8A8>(p, c, err, stream);
-    case kW4A16: return launch_bn<kW4A16>(p, c, err, stream);
+    case kW4A16:
+        return p.interleaved ? launch_bn<kW4A16I>(p, c, err, stream)
+                             : launch_bn<kW4A16>(p, c, err, stream);
     default: return launch_bn<kW2A8>(p, c, err, stream);
     }
 }

@@ -61,7 +61,8 @@ typedef enum qg_op {
     QG_OP_W4A16 = 0,
     QG_OP_W8A8 = 1,
     QG_OP_W2A8 = 2,
-    QG_OP_DENSE_F16 = 3
+    QG_OP_DENSE_F16 = 3,
+    QG_OP_W4A16_INTERLEAVED = 4   /* W4A16 with weights from quant_pack_int4_interleaved */
 } qg_op;
 
 typedef enum qg_path {
@@ -96,6 +97,19 @@ typedef struct qgemm_config_t {
 qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, const void *zeros,
                       void *C, int M, int N, int K, int group_size, int split_k, int has_zero,
                       cudaStream_t stream);
+
+/*
+ * W4A16 with weights in the interleaved (pre-shuffled) layout that quant_pack_int4_interleaved
+ * writes: within each uint32 word the codes k = 8j .. 8j+7 sit in nibbles 0, 4, 1, 5, 2, 6, 3, 7
+ * (nibbles 0..7 hold codes 0, 2, 4, 6, 1, 3, 5, 7), so that the upcast finds codes adjacent in k
+ * in nibbles i and i+4 and needs no byte permutes. Everything else as qgemm_w4a16; the result
+ * is that of qgemm_w4a16 on the naturally packed weights of the same codes, up to the order of
+ * the fp32 additions inside the small-M kernels' MMAs (the tensor-core path gives identical
+ * bits). Configurations are kept under QG_OP_W4A16_INTERLEAVED.
+ */
+qg_status qgemm_w4a16_interleaved(const void *A, const uint32_t *Wq, const void *scales,
+                                  const void *zeros, void *C, int M, int N, int K, int group_size,
+                                  int split_k, int has_zero, cudaStream_t stream);
 
 /*
  * W4A16 with deterministic split-K: the fp32-workspace form of parallel-k (hidet-org/hidet issue
@@ -152,6 +166,15 @@ qg_status qgemm_dense_f16(const void *A, const void *W, void *C, int M, int N, i
  */
 qg_status quant_pack_int4(const uint8_t *codes, uint32_t *packed, int M, int N, int K,
                           int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/*
+ * codes: uint8 [N, K] -> packed: uint32 [N, K/8] in the interleaved layout of
+ * qgemm_w4a16_interleaved: packed[n, j] = sum_e (codes[n, 8j+e] & 0xF) << 4 * pos(e) with
+ * pos = (0, 4, 1, 5, 2, 6, 3, 7). Requires K % 32 == 0. Other arguments as quant_pack_int4.
+ */
+qg_status quant_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int M, int N, int K,
+                                      int group_size, int split_k, int has_zero,
+                                      cudaStream_t stream);
 
 /*
  * vals: int8 [N, K] holding values -2..1 (only the low 2 bits are used) -> packed: uint32
