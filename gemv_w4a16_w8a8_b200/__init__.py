@@ -26,13 +26,17 @@ QG_ERR_CUDA = 4
 QG_ERR_DEVICE_TIMEOUT = 5
 QG_ERR_NOT_SM100 = 6
 QG_ERR_BAD_CONFIG = 7
+QG_ERR_SCRATCH_TOO_SMALL = 8
+# size of the library's fixed device scratch used by qgemm_w4a16_splitk_f32_noalloc
+QGEMM_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 OP_W4A16, OP_W8A8, OP_W2A8, OP_DENSE_F16, OP_W4A16_INTERLEAVED = 0, 1, 2, 3, 4
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 
 # every symbol include/qgemm.h declares
 EXPORTS = (
-    "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes",
+    "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
     "qgemm_version",
@@ -72,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.quant_pack_int4_interleaved.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_w4a16_splitk_f32.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
                                              ctypes.c_size_t, vp]
+        L.qgemm_w4a16_splitk_f32_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                     i32, vp]
         L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.qgemm_w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]

@@ -504,6 +504,82 @@ qg_status quant_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, in
     return QG_OK;
 }
 
+// ---- qgemm_w4a16_splitk_f32_noalloc --------------------------------------------------------------
+// For callers that must not allocate: the deterministic split-K scratch (arrival counters and
+// fp32 partial tiles) lives in this fixed device buffer instead of a caller workspace. Every
+// device that loads the library holds it until exit; all calls on a device share it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QGEMM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};   // device address of g_noalloc_scratch, per device
+}
+
+qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, const void *scales,
+                                         const void *zeros, void *C, int M, int N, int K,
+                                         int group_size, int split_k, int has_zero,
+                                         cudaStream_t stream)
+{
+    qg_status s = check_shape(QG_OP_W4A16, M, N, K, group_size, has_zero, split_k);
+    if (s != QG_OK) return s;
+    if (split_k < 1) return QG_ERR_INVALID_ARG;
+    if (effective_gs(QG_OP_W4A16, K, group_size) % 128) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!A || !Wq || !C || !scales) return QG_ERR_INVALID_ARG;
+    if ((zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(Wq, 16) || !aligned(C, 16) || !aligned(scales, 2) ||
+        (zeros && !aligned(zeros, 2)))
+        return QG_ERR_ALIGNMENT;
+    const size_t need = qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k);
+    if (need == 0) return QG_ERR_INVALID_ARG;
+    if (need > (size_t)QGEMM_NOALLOC_SCRATCH_BYTES) return QG_ERR_SCRATCH_TOO_SMALL;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    void *scratch = nullptr;
+    {
+        // once per device, with that device current: the buffer's device address (in host
+        // code the symbol itself is only a stand-in and must never reach a kernel)
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_ptr[dev]) {
+            void *ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+                cudaGetLastError();
+                return QG_ERR_CUDA;
+            }
+            g_noalloc_ptr[dev] = ptr;
+        }
+        scratch = g_noalloc_ptr[dev];
+    }
+    Problem p = make_problem(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, has_zero);
+    qgemm_config_t c = choose(p, split_k, d->sms);
+    if (c.path != QG_PATH_GEMV || c.stages == 0) {
+        std::memset(&c, 0, sizeof(c));
+        c.path = QG_PATH_GEMV;
+        c.rows = 32;
+        c.stages = 4;
+    }
+    c.split_k = split_k;
+    if (!gemv_w4a16_tma_supports(p, c)) return QG_ERR_BAD_CONFIG;
+    unsigned int *counters = static_cast<unsigned int *>(scratch);
+    float *parts = reinterpret_cast<float *>(static_cast<char *>(scratch) + ws_counter_bytes(M, N));
+    // the arrival counters must start at zero; the partial tiles are overwritten in full
+    if (cudaMemsetAsync(counters, 0, gemv_w4a16_ws_tiles(p, c) * sizeof(unsigned int), stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    if (launch_gemv_w4a16_tma(p, c, d->err_word, stream, parts, counters) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N, int K,
                      int group_size, int split_k, int has_zero, cudaStream_t stream)
 {
@@ -707,6 +783,8 @@ const char *qgemm_status_string(qg_status status)
     case QG_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
     case QG_ERR_NOT_SM100: return "device is not compute capability 10.0 (B200)";
     case QG_ERR_BAD_CONFIG: return "configuration cannot run this problem";
+    case QG_ERR_SCRATCH_TOO_SMALL:
+        return "problem needs more scratch than the library's fixed buffer holds";
     }
     return "unknown status";
 }

@@ -54,7 +54,8 @@ typedef enum qg_status {
     QG_ERR_CUDA = 4,              /* a CUDA runtime call or a kernel launch failed          */
     QG_ERR_DEVICE_TIMEOUT = 5,    /* a kernel gave up a bounded wait (qgemm_sync_check)     */
     QG_ERR_NOT_SM100 = 6,         /* the current device is not compute capability 10.0     */
-    QG_ERR_BAD_CONFIG = 7         /* a config passed to qgemm_set_config cannot run        */
+    QG_ERR_BAD_CONFIG = 7,        /* a config passed to qgemm_set_config cannot run        */
+    QG_ERR_SCRATCH_TOO_SMALL = 8  /* the problem needs more than the fixed scratch buffer   */
 } qg_status;
 
 typedef enum qg_op {
@@ -132,6 +133,31 @@ qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *
 
 /* Workspace bytes qgemm_w4a16_splitk_f32 needs for these arguments (0 if they are invalid). */
 size_t qgemm_w4a16_workspace_bytes(int M, int N, int K, int group_size, int split_k);
+
+/*
+ * qgemm_w4a16_splitk_f32 for callers that cannot allocate device memory: code that runs where
+ * cudaMalloc is not allowed or not wanted (inside a memory pool's or a framework's own
+ * allocator, in a process whose device memory is fully reserved up front, or on a path that
+ * must never block on the allocator). It takes no workspace: the scratch lives in one
+ * statically sized buffer inside the library, QGEMM_NOALLOC_SCRATCH_BYTES bytes of device
+ * memory that every GPU which loads the library holds until the process exits. The source
+ * pages have no counterpart to this entry point.
+ *   - Same arguments and result as qgemm_w4a16_splitk_f32 minus the workspace; the result is
+ *     bit-identical to it.
+ *   - Needs qgemm_w4a16_workspace_bytes(M, N, K, group_size, split_k) <= the buffer size; larger
+ *     problems return QG_ERR_SCRATCH_TOO_SMALL before anything is queued.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call. The first call
+ *     on each device looks up the buffer's device address (cudaGetSymbolAddress, with that
+ *     device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one buffer and leaves its contents behind; each call
+ *     clears the part that must start at zero. Calls that overlap on the GPU (on different
+ *     streams, or from different host threads) race on the buffer: order them.
+ */
+#define QGEMM_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, const void *scales,
+                                         const void *zeros, void *C, int M, int N, int K,
+                                         int group_size, int split_k, int has_zero,
+                                         cudaStream_t stream);
 
 /*
  * W8A8. A: int8 [M, K]. W: int8 [N, K]. C: int32 [M, N] = sum_k A[m,k] * W[n,k], exact
