@@ -31,7 +31,7 @@ QG_ERR_SCRATCH_TOO_SMALL = 8
 QGEMM_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 OP_W4A16, OP_W8A8, OP_W2A8, OP_DENSE_F16, OP_W4A16_INTERLEAVED = 0, 1, 2, 3, 4
-PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_GEMV, PATH_TC, PATH_STREAM = 0, 1, 2, 3
 
 # every symbol include/qgemm.h declares
 EXPORTS = (

@@ -157,6 +157,8 @@ bool supports(const Problem &p, const qgemm_config_t &c)
         return false;
     case QG_PATH_TC:
         return tc_supports(p, c);
+    case QG_PATH_STREAM:
+        return gemv_w4a16_stream_supports(p, c);
     default:
         return false;
     }
@@ -206,11 +208,38 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     return c;
 }
 
-qgemm_config_t heuristic(const Problem &p, int sms)
+// Persistent stream-K W4A16 kernel: 64-row x 512-K stages (256 contiguous bytes of each weight
+// row a copy) consumed by 4 row warps x 2 K warps, in the deepest ring shared memory holds (up
+// to 16 stages: HBM needs ~100 KB in flight per SM), one CTA per SM.
+qgemm_config_t stream_default(const Problem &p)
+{
+    qgemm_config_t c;
+    std::memset(&c, 0, sizeof(c));
+    c.path = QG_PATH_STREAM;
+    c.rows = 16;
+    c.bm = 4;
+    c.bn = 2;
+    c.split_k = 1;
+    for (int bk : {512, 256})
+        for (int st = 16; st >= 2; --st) {
+            c.bk = bk;
+            c.stages = st;
+            if (gemv_w4a16_stream_supports(p, c)) return c;
+        }
+    return c;
+}
+
+qgemm_config_t heuristic(const Problem &p, int sms, bool allow_stream)
 {
     qgemm_config_t c;
     std::memset(&c, 0, sizeof(c));
     c.split_k = 1;
+    // the persistent kernel wins from 9 tokens on (its shared operand table and atomics cost
+    // more than they save below that; both are bound by the warp-level MMA rate)
+    if (allow_stream && p.op == QG_OP_W4A16 && p.M > 8 && p.M <= 16) {
+        qgemm_config_t st = stream_default(p);
+        if (gemv_w4a16_stream_supports(p, st)) return st;
+    }
     // tensor-core GEMM once there are enough tokens to fill its tile
     if (p.op == QG_OP_DENSE_F16 || p.M > 16) {
         qgemm_config_t tc = tc_default(p, sms);
@@ -307,8 +336,12 @@ qgemm_config_t choose(const Problem &p, int split_k, int sms)
             found = true;
         }
     }
-    if (!found) c = heuristic(p, sms);
-    if (split_k > 0) c.split_k = split_k;
+    if (!found) c = heuristic(p, sms, split_k <= 0);
+    if (split_k > 0) {
+        // an explicit split asks for a path that cuts K into exactly that many parts
+        if (c.path == QG_PATH_STREAM) c = heuristic(p, sms, false);
+        c.split_k = split_k;
+    }
     return c;
 }
 
@@ -317,7 +350,7 @@ qgemm_config_t choose(const Problem &p, int split_k, int sms)
 qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStream_t stream)
 {
     if (!supports(p, c)) return QG_ERR_BAD_CONFIG;
-    if (c.split_k > 1) {
+    if (c.split_k > 1 || c.path == QG_PATH_STREAM) {
         if (cudaMemsetAsync(p.C, 0, out_bytes(p), stream) != cudaSuccess) {
             cudaGetLastError();
             return QG_ERR_CUDA;
@@ -334,6 +367,10 @@ qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStre
             e = launch_gemv_int(p, c, stream);
     } else if (c.path == QG_PATH_TC) {
         e = launch_tc(p, c, d->err_word, stream);
+    } else if (c.path == QG_PATH_STREAM) {
+        Problem q = p;
+        q.sms = d->sms;
+        e = launch_gemv_w4a16_stream(q, c, d->err_word, stream);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -382,6 +419,29 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                     c.stages = stage_opts[st];
                     c.split_k = s;
                     if (supports(p, c)) out.push_back(c);
+                }
+    }
+    if (p.op == QG_OP_W4A16 && p.M <= 16) {
+        // every stage shape and warp split, each at its deepest ring and at two-thirds of it
+        qgemm_config_t t = stream_default(p);
+        for (int bk : {256, 512, 1024})
+            for (int wk : {1, 2, 4})
+                for (int wr : {2, 3, 4, 6, 8}) {
+                    t.bk = bk;
+                    t.bn = wk;
+                    t.bm = wr;
+                    int deepest = 0;
+                    for (int st = 2; st <= 16; ++st) {
+                        t.stages = st;
+                        if (supports(p, t)) deepest = st;
+                    }
+                    if (deepest == 0) continue;
+                    t.stages = deepest;
+                    out.push_back(t);
+                    if (deepest * 2 / 3 >= 2 && deepest * 2 / 3 < deepest) {
+                        t.stages = deepest * 2 / 3;
+                        out.push_back(t);
+                    }
                 }
     }
     if (p.op == QG_OP_DENSE_F16 || p.M > 1) {

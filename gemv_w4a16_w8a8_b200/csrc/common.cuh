@@ -23,6 +23,7 @@ struct Problem {
     int gs;        // effective group size (K when the caller passed -1 / 0)
     int has_zero;
     int interleaved = 0;   // W4A16: 1 = codes of each word in nibble order 0,2,4,6,1,3,5,7
+    int sms = 148;         // multiprocessors of the device (persistent grids)
 };
 
 // Launchers return cudaGetLastError() after queueing their kernels on `stream`.
@@ -34,6 +35,9 @@ cudaError_t launch_gemv_w4a16_tma(const Problem &p, const qgemm_config_t &cfg, u
                                   unsigned int *ws_count = nullptr);
 // Arrival counters the deterministic split-K needs (one per output tile of this config).
 size_t gemv_w4a16_ws_tiles(const Problem &p, const qgemm_config_t &cfg);
+// Persistent stream-K W4A16 kernel (path QG_PATH_STREAM); C must be zeroed first.
+cudaError_t launch_gemv_w4a16_stream(const Problem &p, const qgemm_config_t &cfg,
+                                     unsigned int *err, cudaStream_t stream);
 cudaError_t launch_gemv_w2a8_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
                                  cudaStream_t stream);
 cudaError_t launch_gemv_int(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
@@ -49,6 +53,7 @@ cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int 
 // Whether a configuration can run the problem (tile and alignment rules of its kernel).
 bool gemv_w4a16_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &cfg);
+bool gemv_w4a16_stream_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w2a8_tma_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
 bool tc_supports(const Problem &p, const qgemm_config_t &cfg);

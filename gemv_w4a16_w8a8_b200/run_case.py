@@ -4,7 +4,8 @@
 
 Inputs are the seeded synthetic ones. Weights rotate over enough copies that each call reads
 its weights from HBM. Prints the mean device time per call (CUDA events) and the effective
-GB/s and TFLOP/s. --split-k / --rows / --path / --bn / --stages pin a configuration first.
+GB/s and TFLOP/s. --split-k / --rows / --path / --bn / --bk / --bm / --stages pin a
+configuration first.
 """
 from __future__ import annotations
 
@@ -33,6 +34,8 @@ def main(argv=None) -> int:
     ap.add_argument("--rows", type=int, default=0)
     ap.add_argument("--bn", type=int, default=0)
     ap.add_argument("--stages", type=int, default=-1)
+    ap.add_argument("--bk", type=int, default=0)
+    ap.add_argument("--bm", type=int, default=0, help="TC: tile M; STREAM: warps per CTA")
     ap.add_argument("--copies", type=int, default=0, help="weight copies (0: >= 3x L2)")
     a = ap.parse_args(argv)
 
@@ -74,9 +77,13 @@ def main(argv=None) -> int:
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + 2 * M * K + 2 * M * N
 
-    if a.path or a.rows or a.bn or a.stages >= 0:
+    if a.path or a.rows or a.bn or a.bk or a.bm or a.stages >= 0:
         cfg = qg.qgemm_plan(opc, M, N, K, gs, hz)
-        for key, val in (("path", a.path), ("rows", a.rows), ("bn", a.bn), ("split_k", a.split_k)):
+        if a.path and a.path != cfg["path"]:
+            cfg = {k: 0 for k in cfg}
+            cfg["split_k"] = 1
+        for key, val in (("path", a.path), ("rows", a.rows), ("bn", a.bn), ("bk", a.bk),
+                         ("bm", a.bm), ("split_k", a.split_k)):
             if val:
                 cfg[key] = val
         if a.stages >= 0:

@@ -27,7 +27,10 @@
  *     after it started (a bounded wait that ran out) are reported by qgemm_sync_check().
  *   - split_k > 1 makes the call zero C on `stream` first, then add each part into it
  *     atomically; fp16 results then depend on the (unspecified) order of the additions,
- *     int32 results do not. split_k <= 0 selects the tuned or heuristic value for the shape.
+ *     int32 results do not. split_k <= 0 selects the tuned or heuristic value for the shape;
+ *     for W4A16 at M <= 16 that may be the persistent path (QG_PATH_STREAM), which also zeroes
+ *     C and adds partial row blocks atomically. split_k >= 1 keeps to paths that split K into
+ *     exactly that many parts.
  *   - The library allocates no per-call memory. It allocates once per device at first use a
  *     4-byte device error word; qgemm_tune() allocates nothing either (it times the caller's
  *     buffers).
@@ -69,7 +72,15 @@ typedef enum qg_op {
 typedef enum qg_path {
     QG_PATH_AUTO = 0, /* let the library choose                                               */
     QG_PATH_GEMV = 1, /* small-M streaming kernels (weights read once with 128-bit loads)      */
-    QG_PATH_TC = 2    /* tcgen05 tensor-core GEMM with a TMA multi-stage pipeline (large M)   */
+    QG_PATH_TC = 2,   /* tcgen05 tensor-core GEMM with a TMA multi-stage pipeline (large M)   */
+    QG_PATH_STREAM = 3 /* W4A16, M <= 16: persistent grid, every CTA streams an equal run of
+                          (row block, K stage) units through a TMA ring (a copy warp keeps it
+                          full, a prep warp turns the activations into MMA operands); partial
+                          row blocks meet in C through atomics (C is zeroed first). Fields:
+                          rows (16 rows per consumer warp), bk (256, 512 or 1024 K values a
+                          stage), stages (ring depth, 2..16), bm (row warps WR, <= 16), bn (K
+                          warps WK sharing a row block: 1, 2 or 4, dividing bk / 128;
+                          WR * WK <= 14); split_k unused. */
 } qg_path;
 
 /* One launch configuration. Fields a path does not use are ignored (set them to 0). */

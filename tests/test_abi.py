@@ -99,7 +99,14 @@ def test_valid_call_without_gpu_fails_loudly():
 
 def test_plan_small_m_uses_streaming_kernels():
     c = qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1)
+    assert c["path"] == qg.PATH_GEMV and c["rows"] in (16, 32, 64)
+    c = qg.qgemm_plan(qg.OP_W4A16, 12, 4096, 4096, 128, 1)
+    assert c["path"] == qg.PATH_STREAM and c["rows"] == 16 and c["bk"] in (256, 512, 1024)
+    # K not a multiple of 256 leaves the persistent kernel for the split-K streaming kernels
+    c = qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4224, 128, 1)
     assert c["path"] == qg.PATH_GEMV and c["split_k"] >= 1 and c["rows"] in (16, 32, 64)
+    c = qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1, split_k=2)
+    assert c["path"] == qg.PATH_GEMV and c["split_k"] == 2
     c = qg.qgemm_plan(qg.OP_W8A8, 1, 16384, 16384)
     assert c["path"] == qg.PATH_GEMV and c["rows"] in (1, 2, 4, 8)
     c = qg.qgemm_plan(qg.OP_W2A8, 1, 16384, 16384)
@@ -110,6 +117,34 @@ def test_plan_split_override():
     assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1, split_k=4)["split_k"] == 4
     with pytest.raises(qg.QGemmError):
         qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 100, 1)
+
+
+def test_stream_config_rules():
+    ok = {"path": qg.PATH_STREAM, "rows": 16, "bm": 4, "bn": 2, "bk": 512, "stages": 10,
+          "split_k": 1, "swap_ab": 0}
+    qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 4096, 128, 1, ok)
+    try:
+        assert qg.qgemm_plan(qg.OP_W4A16, 1, 4096, 4096, 128, 1) == ok
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 4096, 128, 1, None)
+    bad = [dict(ok, rows=32), dict(ok, bk=2048), dict(ok, stages=16),   # 304 KB of ring
+           dict(ok, bn=3), dict(ok, bn=8), dict(ok, bk=256, bn=4),    # 2 sub-blocks, 4 K warps
+           dict(ok, bm=8), dict(ok, bm=0), dict(ok, stages=1), dict(ok, stages=17)]
+    for cfg in bad:
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 4096, 128, 1, cfg)
+    # the activations' share of shared memory grows with M
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, 16, 4096, 4096, 128, 1, ok)
+    # the persistent kernel covers M <= 16 and K a multiple of 256 only
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, 17, 4096, 4096, 128, 1, dict(ok, stages=4))
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, 4, 4096, 4224, 128, 1, dict(ok, stages=4))
+    # the default plan fits at every M the heuristic gives the path
+    for M in range(9, 17):
+        c = qg.qgemm_plan(qg.OP_W4A16, M, 16384, 16384, 128, 1)
+        assert c["path"] == qg.PATH_STREAM, (M, c)
 
 
 def test_set_save_load_roundtrip(tmp_path):
