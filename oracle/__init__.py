@@ -43,6 +43,9 @@ class Oracle:
             getattr(L, name).argtypes = [_ptr, _ptr, _i64, _i64]
             getattr(L, name).restype = ctypes.c_int
         L.orc_decode_half.argtypes = [_ptr, _ptr, _i64]
+        L.orc_float_to_half.argtypes = [ctypes.c_float]
+        L.orc_float_to_half.restype = ctypes.c_uint16
+        L.orc_rtn_int4.argtypes = [_ptr, _i64, _i64, _i64, _ptr, _ptr, _ptr]
         L.orc_w4a16.argtypes = [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, ctypes.c_int,
                                 _ptr, ctypes.c_int]
         L.orc_w4a16_at.argtypes = [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, ctypes.c_int,
@@ -74,6 +77,26 @@ class Oracle:
         out = np.empty(b.shape, dtype=np.float64)
         self.L.orc_decode_half(_p(b), _p(out), b.size)
         return out
+
+    def float_to_half(self, x: np.ndarray) -> np.ndarray:
+        """binary16 bits of each float32 value, round to nearest even."""
+        x = np.ascontiguousarray(x, dtype=np.float32).ravel()
+        out = np.empty(x.size, dtype=np.uint16)
+        for i, v in enumerate(x):
+            out[i] = self.L.orc_float_to_half(ctypes.c_float(float(v)))
+        return out
+
+    def rtn_int4(self, W, group_size: int):
+        """Round-to-nearest int4 quantisation of fp16 W [N, K]: (codes u8 [N, K], scales fp16
+        [N, G], zeros fp16 [N, G])."""
+        Wb = _bits16(W)
+        N, K = Wb.shape
+        gs = K if group_size <= 0 else group_size
+        codes = np.empty((N, K), dtype=np.uint8)
+        S = np.empty((N, K // gs), dtype=np.uint16)
+        Z = np.empty((N, K // gs), dtype=np.uint16)
+        _check(self.L.orc_rtn_int4(_p(Wb), N, K, group_size, _p(codes), _p(S), _p(Z)), "rtn_int4")
+        return codes, S.view(np.float16), Z.view(np.float16)
 
     def pack_int4(self, codes: np.ndarray) -> np.ndarray:
         codes = np.ascontiguousarray(codes, dtype=np.uint8)
@@ -235,6 +258,8 @@ def get() -> Oracle:
 
 def max_threads() -> int: return get().max_threads()
 def half_to_double(b): return get().half_to_double(b)
+def float_to_half(x): return get().float_to_half(x)
+def rtn_int4(W, group_size): return get().rtn_int4(W, group_size)
 def pack_int4(c): return get().pack_int4(c)
 def unpack_int4(p, K): return get().unpack_int4(p, K)
 def pack_int4_interleaved(c): return get().pack_int4_interleaved(c)

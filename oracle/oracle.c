@@ -401,6 +401,84 @@ int orc_w2a8_at(const int8_t *A, const uint32_t *Wq, int64_t M, int64_t N, int64
     return int_gemm_at(A, Wq, 2, M, N, K, ms, ns, count, out, nthreads);
 }
 
+/* IEEE 754 binary16 encoding of a binary32 value, round to nearest, ties to even; overflow
+   to infinity, NaN to a quiet NaN. Built from the two formats' definitions: a float is
+   m * 2^(E-23) with m the 24-bit significand; a half keeps 11 significant bits when
+   E >= -14 and a fixed 2^-24 unit below that. */
+uint16_t orc_float_to_half(float x)
+{
+    uint32_t b;
+    memcpy(&b, &x, sizeof b);
+    const uint16_t sign = (uint16_t)((b >> 16) & 0x8000u);
+    const uint32_t e = (b >> 23) & 0xFFu, f = b & 0x7FFFFFu;
+    if (e == 0xFFu) return (uint16_t)(sign | 0x7C00u | (f ? 0x200u : 0u));
+    if (e == 0) return sign;                  /* below 2^-126: far under half a half-ulp */
+    const int32_t E = (int32_t)e - 127;
+    if (E > 15) return (uint16_t)(sign | 0x7C00u);
+    const uint32_t m = 0x800000u | f;
+    const int shift = E >= -14 ? 13 : 13 + (-14 - E);   /* significand bits that go */
+    if (shift > 24) return sign;
+    uint32_t q = m >> shift;
+    const uint32_t rem = m & ((1u << shift) - 1u), halfway = 1u << (shift - 1);
+    if (rem > halfway || (rem == halfway && (q & 1u))) ++q;
+    if (E >= -14) {
+        uint32_t he = (uint32_t)(E + 15);
+        if (q == 2048u) {                      /* rounding carried into the exponent */
+            q = 1024u;
+            ++he;
+        }
+        if (he >= 31u) return (uint16_t)(sign | 0x7C00u);
+        return (uint16_t)(sign | (he << 10) | (q & 0x3FFu));
+    }
+    return (uint16_t)(sign | q);               /* subnormal (q == 1024 encodes 2^-14) */
+}
+
+/* Round-to-nearest int4 quantisation of fp16 weights W [N, K] into codes [N, K] (0..15) and
+   fp16 scales / zeros [N, K / group_size], such that w ~ (q - z) * s.
+   Source: the torchao issue's workflow table names int4 weight-only quantisation
+   (Int4WeightOnlyConfig) without a formula; the reading used here (design notes):
+   asymmetric min-max per group with the range widened to include 0,
+       lo = min(0, min w), hi = max(0, max w), s = fp16((hi - lo) / 15)  (1 if hi == lo;
+       the smallest subnormal if it rounds to 0), z = clamp(rint(0 - lo / s), 0, 15),
+       q = clamp(rint(w / s) + z, 0, 15),
+   rint rounding half to even. The values that decide a code (hi - lo, the divisions, rint)
+   are evaluated in binary32 because the kernels decide in binary32 too. */
+int orc_rtn_int4(const uint16_t *W, int64_t N, int64_t K, int64_t group_size, uint8_t *codes,
+                 uint16_t *S, uint16_t *Z)
+{
+    const int64_t gs = (group_size <= 0) ? K : group_size;
+    if (N <= 0 || K <= 0 || gs <= 0 || K % gs) return ORC_BAD_ARGS;
+    const int64_t G = K / gs;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            const uint16_t *w = W + n * K + g * gs;
+            float lo = 0.0f, hi = 0.0f;
+            for (int64_t k = 0; k < gs; ++k) {
+                const float v = (float)orc_half_to_double(w[k]);   /* exact */
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            const float range = hi - lo;
+            const float s32 = range > 0.0f ? range / 15.0f : 1.0f;
+            uint16_t s16 = orc_float_to_half(s32);
+            if ((s16 & 0x7FFFu) == 0) s16 = 0x0001u;
+            const float s = (float)orc_half_to_double(s16);
+            float z = rintf(0.0f - lo / s);    /* +0, not -0, when lo is 0 */
+            if (z < 0.0f) z = 0.0f;
+            if (z > 15.0f) z = 15.0f;
+            S[n * G + g] = s16;
+            Z[n * G + g] = orc_float_to_half(z);
+            for (int64_t k = 0; k < gs; ++k) {
+                const float v = (float)orc_half_to_double(w[k]);
+                float q = rintf(v / s) + z;
+                if (q < 0.0f) q = 0.0f;
+                if (q > 15.0f) q = 15.0f;
+                codes[n * K + g * gs + k] = (uint8_t)q;
+            }
+        }
+    return ORC_OK;
+}
+
 int orc_max_threads(void)
 {
 #ifdef _OPENMP

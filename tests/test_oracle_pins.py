@@ -317,6 +317,119 @@ def test_fp16_close_rule():
     assert not oracle.fp16_close(nan, ref)[0]
 
 
+# ---- fp16 encoding and round-to-nearest int4 quantisation ------------------------------------------
+
+def check_float_to_half(orc):
+    """Against numpy's float32 -> float16 conversion (round to nearest even): every float16 value,
+    the midpoints between neighbours (ties), values just off them, subnormals and overflow."""
+    rng = np.random.default_rng(3)
+    halves = np.arange(0, 0x7C00, 97, dtype=np.uint16).view(np.float16)
+    exact = halves.astype(np.float32)
+    nxt = np.nextafter(halves, np.float16(np.inf)).astype(np.float32)
+    mids = ((exact.astype(np.float64) + nxt.astype(np.float64)) / 2).astype(np.float32)
+    off = np.concatenate([np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9))])
+    rand = (rng.standard_normal(2000) * np.exp2(rng.integers(-26, 17, 2000))).astype(np.float32)
+    edge = np.array([0.0, -0.0, 65504.0, 65519.9, 65520.0, 1e9, 2.0**-24, 2.0**-25, 3 * 2.0**-26,
+                     2.0**-26, -2.0**-14, np.inf, -np.inf], dtype=np.float32)
+    xs = np.concatenate([exact, mids, off, rand, -rand, edge])
+    got = orc.float_to_half(xs)
+    want = xs.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:5]
+    assert (orc.float_to_half(np.array([np.nan], np.float32))[0] & 0x7C00) == 0x7C00
+
+
+def test_float_to_half_matches_numpy():
+    check_float_to_half(oracle.get())
+
+
+def _rtn_fixture():
+    path = os.path.join(os.path.dirname(__file__), "golden", "rtn_int4.txt")
+    gs, rows = None, []
+    with open(path) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            key, *vals = line.split()
+            if key == "gs":
+                gs = int(vals[0])
+            elif key == "row":
+                rows.append({})
+            elif key == "w":
+                rows[-1]["w"] = np.array([float(v) for v in vals], dtype=np.float16)
+            elif key == "q":
+                rows[-1]["q"] = np.array([int(v) for v in vals], dtype=np.uint8)
+            else:
+                rows[-1][key] = np.array([int(v, 16) for v in vals], dtype=np.uint16)
+    return gs, rows
+
+
+def check_rtn_golden(orc):
+    gs, rows = _rtn_fixture()
+    for r in rows:
+        codes, S, Z = orc.rtn_int4(r["w"][None, :], gs)
+        assert np.array_equal(codes[0], r["q"]), (codes[0], r["q"])
+        assert np.array_equal(S[0].view(np.uint16), r["s"]), S[0].view(np.uint16)
+        assert np.array_equal(Z[0].view(np.uint16), r["z"]), Z[0].view(np.uint16)
+
+
+def test_rtn_golden_fixture():
+    check_rtn_golden(oracle.get())
+
+
+def check_rtn_error_bound(orc):
+    """(q - z) s is within s/2 of w wherever the code is not clamped, within s everywhere; the
+    group's extreme values take the codes 0 and 15 whenever the group straddles 0."""
+    rng = np.random.default_rng(5)
+    N, K, gs = 64, 512, 128
+    W = (rng.standard_normal((N, K)) * np.exp2(rng.integers(-6, 4, (N, 1)))).astype(np.float16)
+    W[:8] = np.abs(W[:8])          # all-positive rows
+    W[8:16] = -np.abs(W[8:16])     # all-negative rows
+    codes, S, Z = orc.rtn_int4(W, gs)
+    s = np.repeat(S.astype(np.float64), gs, axis=1)
+    z = np.repeat(Z.astype(np.float64), gs, axis=1)
+    err = np.abs(W.astype(np.float64) - (codes.astype(np.float64) - z) * s)
+    inner = (codes > 0) & (codes < 15)
+    assert np.all(err[inner] <= 0.5 * s[inner] * (1 + 1e-6))
+    assert np.all(err <= s * (1 + 1e-6))
+    assert codes.max() <= 15 and np.all(Z.astype(np.float64) == np.rint(Z.astype(np.float64)))
+    g = W.reshape(N, K // gs, gs).astype(np.float64)
+    c = codes.reshape(N, K // gs, gs)
+    straddle = (g.min(axis=2) < 0) & (g.max(axis=2) > 0)
+    lo_code = np.take_along_axis(c, g.argmin(axis=2)[..., None], axis=2)[..., 0]
+    hi_code = np.take_along_axis(c, g.argmax(axis=2)[..., None], axis=2)[..., 0]
+    assert np.all(lo_code[straddle] == 0) and np.all(hi_code[straddle] >= 14)
+
+
+def test_rtn_error_bound():
+    check_rtn_error_bound(oracle.get())
+
+
+def check_rtn_closed_forms(orc):
+    """Constant groups: 0 -> (s 1, z 0, q 0); c > 0 -> (s = c/15, z 0, q 15); c < 0 ->
+    (s = -c/15, z 15, q 0). Scaling W by 2 doubles s exactly and keeps codes and zeros."""
+    gs = 32
+    W = np.concatenate([np.zeros(gs), np.full(gs, 3.0), np.full(gs, -1.5)]).astype(np.float16)
+    codes, S, Z = orc.rtn_int4(W[None, :], gs)
+    assert np.array_equal(codes[0], np.repeat(np.array([0, 15, 0], np.uint8), gs))
+    assert np.array_equal(S[0].astype(np.float64),
+                          np.array([1.0, np.float16(np.float32(3.0) / np.float32(15.0)),
+                                    np.float16(np.float32(1.5) / np.float32(15.0))]))
+    assert np.array_equal(Z[0].astype(np.float64), np.array([0.0, 0.0, 15.0]))
+    rng = np.random.default_rng(6)
+    W = (rng.standard_normal((16, 256))).astype(np.float16)
+    c1, s1, z1 = orc.rtn_int4(W, 64)
+    c2, s2, z2 = orc.rtn_int4((W.astype(np.float32) * 2).astype(np.float16), 64)
+    assert np.array_equal(c1, c2) and np.array_equal(z1, z2)
+    assert np.array_equal(s2.astype(np.float64), 2 * s1.astype(np.float64))
+    # one group spanning K equals group_size = K
+    assert all(np.array_equal(a, b) for a, b in zip(orc.rtn_int4(W, -1), orc.rtn_int4(W, 256)))
+
+
+def test_rtn_closed_forms():
+    check_rtn_closed_forms(oracle.get())
+
+
 # ---- mutation check: each plausible mistake fails at least one pin ------------------------------------
 
 MUTANTS = [
@@ -346,13 +459,23 @@ MUTANTS = [
     ("interleaved unpack shift", "(4 * ILV_POS[k % 8])) & 0xF)", "(4 * (k % 8))) & 0xF)"),
     ("int2 pack not masked", "((uint8_t)vals[n * K + 16 * j + i] & 3u)",
      "((uint8_t)vals[n * K + 16 * j + i])"),
+    ("half encoding ties away from zero", "(rem == halfway && (q & 1u))", "(rem == halfway)"),
+    ("half encoding drops the exponent carry", "q = 1024u;\n            ++he;", "q = 1023u;"),
+    ("rtn truncates", "float q = rintf(v / s) + z;", "float q = truncf(v / s) + z;"),
+    ("rtn range not widened to 0", "float lo = 0.0f, hi = 0.0f;",
+     "float lo = (float)orc_half_to_double(w[0]), hi = lo;"),
+    ("rtn zero sign", "float z = rintf(0.0f - lo / s);", "float z = rintf(lo / s);"),
+    ("rtn sixteen steps", "range / 15.0f", "range / 16.0f"),
+    ("rtn scale not rounded to fp16", "const float s = (float)orc_half_to_double(s16);",
+     "const float s = s32;"),
 ]
 
 PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
         check_w4_one_hot_reads_single_weight, check_w4_constant_closed_form,
         check_w4_per_channel_equals_one_group, check_w4_parallel_k_additivity,
         check_w4_elementwise_matches_full, check_dense_is_numpy_matmul,
-        check_w8a8_is_integer_matmul, check_w2a8_is_integer_matmul]
+        check_w8a8_is_integer_matmul, check_w2a8_is_integer_matmul, check_float_to_half,
+        check_rtn_golden, check_rtn_error_bound, check_rtn_closed_forms]
 
 
 def _build_mutant(src: str, tmpdir: str, idx: int):
