@@ -37,6 +37,7 @@ PATH_AUTO, PATH_GEMV, PATH_TC, PATH_STREAM = 0, 1, 2, 3
 EXPORTS = (
     "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes",
     "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "quant_rtn_int4",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
     "qgemm_version",
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
                                              ctypes.c_size_t, vp]
         L.qgemm_w4a16_splitk_f32_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                      i32, vp]
+        L.quant_rtn_int4.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.qgemm_w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
@@ -294,6 +296,23 @@ def quant_pack_int4(codes, out=None, stream=None):
     _check(lib().quant_pack_int4(_ptr(codes), _ptr(out), 0, N, K, -1, 1, 0, _stream(stream)),
            "quant_pack_int4")
     return out
+
+
+def quant_rtn_int4(W, group_size: int = 128, stream=None):
+    """Round-to-nearest int4 quantisation of fp16 W [N,K] (rule in include/qgemm.h):
+    returns (packed int32 [N,K/8], scales fp16 [N,G], zeros fp16 [N,G])."""
+    torch = _torch()
+    _need(W, torch.float16, 2, "W")
+    N, K = W.shape
+    gs = K if group_size <= 0 else group_size
+    if gs <= 0 or K % gs:
+        raise ValueError(f"group_size {group_size} does not divide K = {K}")
+    Wq = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+    S = torch.empty((N, K // gs), dtype=torch.float16, device=W.device)
+    Z = torch.empty((N, K // gs), dtype=torch.float16, device=W.device)
+    _check(lib().quant_rtn_int4(_ptr(W), _ptr(Wq), _ptr(S), _ptr(Z), N, K, group_size, 1,
+                                _stream(stream)), "quant_rtn_int4")
+    return Wq, S, Z
 
 
 def quant_pack_int2(vals, out=None, stream=None):

@@ -677,6 +677,28 @@ qg_status quant_pack_int4(const uint8_t *codes, uint32_t *packed, int M, int N, 
     return QG_OK;
 }
 
+qg_status quant_rtn_int4(const void *W, uint32_t *Wq, void *scales, void *zeros, int N, int K,
+                         int group_size, int has_zero, cudaStream_t stream)
+{
+    if (!W || !Wq || !scales || N <= 0 || K <= 0 || group_size < -1) return QG_ERR_INVALID_ARG;
+    if (has_zero != 1 || !zeros) return QG_ERR_INVALID_ARG;   // unsigned codes need the zero point
+    if (K % 32) return QG_ERR_UNSUPPORTED_SHAPE;
+    const int gs = group_size <= 0 ? K : group_size;
+    if (K % gs || !(gs == 32 || gs == 64 || gs == 128 || gs % 256 == 0))
+        return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(W, 16) || !aligned(Wq, 16) || !aligned(scales, 2) || !aligned(zeros, 2))
+        return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_rtn_int4(static_cast<const __half *>(W), Wq, static_cast<__half *>(scales),
+                        static_cast<__half *>(zeros), N, K, gs, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 qg_status quant_pack_int2(const int8_t *vals, uint32_t *packed, int M, int N, int K,
                           int group_size, int split_k, int has_zero, cudaStream_t stream)
 {

@@ -45,6 +45,9 @@ cudaError_t launch_pack_int4(const uint8_t *codes, uint32_t *packed, int N, int 
                              cudaStream_t stream);
 cudaError_t launch_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int N, int K,
                                          cudaStream_t stream);
+// Round-to-nearest int4 quantisation (group size 32, 64, 128 or a multiple of 256 dividing K).
+cudaError_t launch_rtn_int4(const __half *W, uint32_t *Wq, __half *S, __half *Z, int N, int K,
+                            int gs, cudaStream_t stream);
 cudaError_t launch_pack_int2(const int8_t *vals, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
 cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int *err_word,

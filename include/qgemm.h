@@ -196,6 +196,26 @@ qg_status qgemm_dense_f16(const void *A, const void *W, void *C, int M, int N, i
 /* ---- weight packing ------------------------------------------------------------------------ */
 
 /*
+ * Round-to-nearest int4 quantisation of fp16 weights W [N, K] into packed codes Wq [N, K/8]
+ * (the layout of quant_pack_int4) and fp16 scales, zeros [N, K/group_size], so that
+ * qgemm_w4a16 with these operands computes A . W~^T for the quantised W~ = (q - z) * s.
+ * The pytorch/ao issue's workflow table names int4 weight-only quantisation
+ * (Int4WeightOnlyConfig) without a formula; the rule implemented, per group of group_size
+ * consecutive K values of a row:
+ *     lo = min(0, min w), hi = max(0, max w),
+ *     s  = fp16_rn((hi - lo) / 15)   (1 when hi == lo; the smallest subnormal if it rounds to 0)
+ *     z  = clamp(rint(0 - lo / s), 0, 15),   q = clamp(rint(w / s) + z, 0, 15),
+ * rint rounding half to even; the divisions and rint are binary32 operations (correctly
+ * rounded). So |w - (q - z) s| <= s / 2 wherever q is not clamped.
+ *   - has_zero must be 1 and zeros non-NULL (unsigned codes need the zero point).
+ *   - group_size: 32, 64, 128 or a multiple of 256 dividing K; -1 / 0 for one group over K.
+ *   - Requires K % 32 == 0; W and Wq 16-byte aligned, scales and zeros 2-byte aligned.
+ *   - Weights are expected finite.
+ */
+qg_status quant_rtn_int4(const void *W, uint32_t *Wq, void *scales, void *zeros, int N, int K,
+                         int group_size, int has_zero, cudaStream_t stream);
+
+/*
  * codes: uint8 [N, K] (only the low 4 bits are used) -> packed: uint32 [N, K/8],
  *     packed[n, j] = sum_{i<8} (codes[n, 8j+i] & 0xF) << 4i.
  * M, group_size, split_k and has_zero are accepted for a uniform call shape and ignored.
