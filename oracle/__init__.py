@@ -46,6 +46,7 @@ class Oracle:
         L.orc_float_to_half.argtypes = [ctypes.c_float]
         L.orc_float_to_half.restype = ctypes.c_uint16
         L.orc_rtn_int4.argtypes = [_ptr, _i64, _i64, _i64, _ptr, _ptr, _ptr]
+        L.orc_w8a8_requant.argtypes = [_ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, ctypes.c_int]
         L.orc_w4a16.argtypes = [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, ctypes.c_int,
                                 _ptr, ctypes.c_int]
         L.orc_w4a16_at.argtypes = [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _i64, ctypes.c_int,
@@ -97,6 +98,20 @@ class Oracle:
         Z = np.empty((N, K // gs), dtype=np.uint16)
         _check(self.L.orc_rtn_int4(_p(Wb), N, K, group_size, _p(codes), _p(S), _p(Z)), "rtn_int4")
         return codes, S.view(np.float16), Z.view(np.float16)
+
+    def w8a8_requant(self, A, W, mult, nthreads=None):
+        """int8 [M, N]: the int32 product of A and W times mult[n], rounded half to even and
+        saturated (binary32 arithmetic)."""
+        A = np.ascontiguousarray(A, dtype=np.int8)
+        W = np.ascontiguousarray(W, dtype=np.int8)
+        mult = np.ascontiguousarray(mult, dtype=np.float32)
+        M, K = A.shape
+        N = W.shape[0]
+        assert W.shape == (N, K) and mult.shape == (N,)
+        C8 = np.empty((M, N), dtype=np.int8)
+        _check(self.L.orc_w8a8_requant(_p(A), _p(W), _p(mult), M, N, K, _p(C8),
+                                       self._threads(nthreads)), "w8a8_requant")
+        return C8
 
     def pack_int4(self, codes: np.ndarray) -> np.ndarray:
         codes = np.ascontiguousarray(codes, dtype=np.uint8)
@@ -258,6 +273,7 @@ def get() -> Oracle:
 
 def max_threads() -> int: return get().max_threads()
 def half_to_double(b): return get().half_to_double(b)
+def w8a8_requant(A, W, mult, nthreads=None): return get().w8a8_requant(A, W, mult, nthreads)
 def float_to_half(x): return get().float_to_half(x)
 def rtn_int4(W, group_size): return get().rtn_int4(W, group_size)
 def pack_int4(c): return get().pack_int4(c)

@@ -479,6 +479,36 @@ int orc_rtn_int4(const uint16_t *W, int64_t N, int64_t K, int64_t group_size, ui
     return ORC_OK;
 }
 
+/* W8A8 with int8 requantised output: C8[m, n] = clamp(rint(float(C[m, n]) * mult[n]), -128,
+   127) with C the exact int32 product of orc_w8a8.
+   Source: microsoft/BitBLAS issue #252, benchmark configuration listing: the int8 x int8
+   configurations carry an int8 output type besides the int32 accumulator. The pages do not say
+   how the accumulator becomes int8; the reading (design notes) is a per-output-channel binary32
+   multiplier, round half to even, saturation. The conversion, the product and rint are binary32
+   operations because the kernels decide in binary32 too. */
+int orc_w8a8_requant(const int8_t *A, const int8_t *W, const float *mult, int64_t M, int64_t N,
+                     int64_t K, int8_t *C8, int nthreads)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || K > 131072) return ORC_BAD_ARGS;
+    int64_t *acc = (int64_t *)malloc((size_t)(M * N) * sizeof(int64_t));
+    if (!acc) return ORC_NO_MEMORY;
+    const int rc = orc_w8a8(A, W, M, N, K, acc, nthreads);
+    if (rc != ORC_OK) {
+        free(acc);
+        return rc;
+    }
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            const float x = (float)(int32_t)acc[m * N + n] * mult[n];
+            float r = rintf(x);
+            if (r < -128.0f) r = -128.0f;
+            if (r > 127.0f) r = 127.0f;
+            C8[m * N + n] = (int8_t)r;
+        }
+    free(acc);
+    return ORC_OK;
+}
+
 int orc_max_threads(void)
 {
 #ifdef _OPENMP

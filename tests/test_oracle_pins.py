@@ -430,6 +430,39 @@ def test_rtn_closed_forms():
     check_rtn_closed_forms(oracle.get())
 
 
+# ---- W8A8 with int8 requantised output ---------------------------------------------------------------
+
+def check_w8a8_requant(orc):
+    """Closed forms on hand-built operands: with one-hot activations C[m, n] = W[n, k]; a
+    multiplier of 1 returns it, 0.5 halves it with ties to even (W odd -> x.5), 4 saturates at
+    both ends, and the multiplier is indexed by the output channel n."""
+    K = 16
+    W = np.array([[-128, -7, -5, -3, -1, 0, 1, 3, 5, 7, 9, 31, 33, 63, 64, 127]], np.int8).T
+    W = np.repeat(W, K, axis=1)                       # row n is the constant W[n]
+    A = np.zeros((1, K), np.int8)
+    A[0, 5] = 1                                        # one-hot: C[0, n] = W[n, 5] = W[n]
+    w = W[:, 0].astype(np.int64)
+    N = W.shape[0]
+    assert np.array_equal(orc.w8a8_requant(A, W, np.ones(N, np.float32))[0], w)
+    half = orc.w8a8_requant(A, W, np.full(N, 0.5, np.float32))[0].astype(np.int64)
+    want = np.array([-64, -4, -2, -2, 0, 0, 0, 2, 2, 4, 4, 16, 16, 32, 32, 64])   # ties to even
+    assert np.array_equal(half, want), half
+    four = orc.w8a8_requant(A, W, np.full(N, 4.0, np.float32))[0].astype(np.int64)
+    assert np.array_equal(four, np.clip(4 * w, -128, 127))
+    mult = np.arange(N, dtype=np.float32) / 16
+    got = orc.w8a8_requant(A, W, mult)[0].astype(np.int64)
+    assert np.array_equal(got, np.clip(np.rint(w.astype(np.float32) * mult), -128, 127))
+    # a large accumulator: A = W = -128 over K = 256 gives 4194304, times 2^-15 = 128 -> 127
+    A2 = np.full((1, 256), -128, np.int8)
+    W2 = np.full((2, 256), -128, np.int8)
+    out = orc.w8a8_requant(A2, W2, np.array([2.0**-15, -2.0**-15], np.float32))[0]
+    assert out.tolist() == [127, -128]
+
+
+def test_w8a8_requant_closed_forms():
+    check_w8a8_requant(oracle.get())
+
+
 # ---- mutation check: each plausible mistake fails at least one pin ------------------------------------
 
 MUTANTS = [
@@ -468,6 +501,9 @@ MUTANTS = [
     ("rtn sixteen steps", "range / 15.0f", "range / 16.0f"),
     ("rtn scale not rounded to fp16", "const float s = (float)orc_half_to_double(s16);",
      "const float s = s32;"),
+    ("requant rounds half away", "float r = rintf(x);", "float r = roundf(x);"),
+    ("requant saturates asymmetrically", "if (r < -128.0f) r = -128.0f;", "if (r < -127.0f) r = -127.0f;"),
+    ("requant multiplier by row", "* mult[n];", "* mult[m];"),
 ]
 
 PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
@@ -475,7 +511,7 @@ PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved, check_p
         check_w4_per_channel_equals_one_group, check_w4_parallel_k_additivity,
         check_w4_elementwise_matches_full, check_dense_is_numpy_matmul,
         check_w8a8_is_integer_matmul, check_w2a8_is_integer_matmul, check_float_to_half,
-        check_rtn_golden, check_rtn_error_bound, check_rtn_closed_forms]
+        check_rtn_golden, check_rtn_error_bound, check_rtn_closed_forms, check_w8a8_requant]
 
 
 def _build_mutant(src: str, tmpdir: str, idx: int):
