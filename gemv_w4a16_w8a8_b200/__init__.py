@@ -37,7 +37,7 @@ PATH_AUTO, PATH_GEMV, PATH_TC, PATH_STREAM = 0, 1, 2, 3
 EXPORTS = (
     "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes",
     "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
-    "quant_rtn_int4",
+    "quant_rtn_int4", "qgemm_w8a8_requant",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
     "qgemm_version",
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.qgemm_w4a16_splitk_f32_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                                      i32, vp]
         L.quant_rtn_int4.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.qgemm_w8a8_requant.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.qgemm_w4a16_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
@@ -251,6 +252,23 @@ def qgemm_w8a8(A, W, C=None, split_k: int = 0, stream=None):
     _need(C, torch.int32, 2, "C")
     _check(lib().qgemm_w8a8(_ptr(A), _ptr(W), _ptr(C), M, N, K, -1, split_k, 0, _stream(stream)),
            "qgemm_w8a8")
+    return C
+
+
+def qgemm_w8a8_requant(A, W, mult, C=None, stream=None):
+    """int8 A [M,K] x int8 W [N,K] -> int8 C [M,N] = sat8(rint(acc * mult[n])), mult fp32 [N]."""
+    torch = _torch()
+    _need(A, torch.int8, 2, "A")
+    _need(W, torch.int8, 2, "W")
+    _need(mult, torch.float32, 1, "mult")
+    M, K = A.shape
+    N = W.shape[0]
+    if W.shape[1] != K or mult.shape[0] != N:
+        raise ValueError("shapes of A, W and mult do not agree")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.int8, device=A.device)
+    _check(lib().qgemm_w8a8_requant(_ptr(A), _ptr(W), _ptr(mult), _ptr(C), M, N, K,
+                                    _stream(stream)), "qgemm_w8a8_requant")
     return C
 
 

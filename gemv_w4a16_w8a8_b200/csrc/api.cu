@@ -647,6 +647,24 @@ qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N,
                   stream);
 }
 
+qg_status qgemm_w8a8_requant(const int8_t *A, const int8_t *W, const float *mult, int8_t *C,
+                             int M, int N, int K, cudaStream_t stream)
+{
+    qg_status s = check_shape(QG_OP_W8A8, M, N, K, -1, 0, 1);
+    if (s != QG_OK) return s;
+    if (!A || !W || !mult || !C) return QG_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(W, 16) || !aligned(mult, 4)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    Problem p = make_problem(QG_OP_W8A8, A, W, nullptr, nullptr, C, M, N, K, -1, 0);
+    p.mult = mult;
+    // rounding needs the whole sum: one K part, never atomics
+    qgemm_config_t c = choose(p, 1, d->sms);
+    if (c.split_k != 1 || !supports(p, c)) return QG_ERR_BAD_CONFIG;
+    return run(p, c, d, stream);
+}
+
 qg_status qgemm_w2a8(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int N, int K,
                      int group_size, int split_k, int has_zero, cudaStream_t stream)
 {

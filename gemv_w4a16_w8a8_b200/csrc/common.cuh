@@ -24,7 +24,16 @@ struct Problem {
     int has_zero;
     int interleaved = 0;   // W4A16: 1 = codes of each word in nibble order 0,2,4,6,1,3,5,7
     int sms = 148;         // multiprocessors of the device (persistent grids)
+    const float *mult = nullptr;   // W8A8: per-channel multiplier -> int8 output (else int32)
 };
+
+// int8 requantisation of an exact int32 accumulator: clamp(rint(float(v) * m), -128, 127),
+// every step a correctly rounded binary32 operation.
+__device__ __forceinline__ int8_t requant_i8(int v, float m)
+{
+    const float r = rintf(__fmul_rn(__int2float_rn(v), m));
+    return (int8_t)(int)fminf(fmaxf(r, -128.0f), 127.0f);
+}
 
 // Launchers return cudaGetLastError() after queueing their kernels on `stream`.
 cudaError_t launch_gemv_w4a16(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);

@@ -47,7 +47,7 @@ template <int R, int MT, bool INT2>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_int_kernel(const int8_t *__restrict__ A, const uint8_t *__restrict__ W,
                 int32_t *__restrict__ C, int M, int N, int K, int chunks_per_split,
-                int atomic_out)
+                int atomic_out, const float *__restrict__ mult)
 {
     constexpr int KC = INT2 ? 64 : 16;           // K values per 16-byte weight chunk
     const int lane = threadIdx.x & 31;
@@ -156,9 +156,10 @@ gemv_int_kernel(const int8_t *__restrict__ A, const uint8_t *__restrict__ W,
         for (int r = 0; r < R; ++r) {
             const int v = warp_sum(acc[r][t]) - corr;
             if (lane == 0 && wok[r] && aok[t]) {
-                int32_t *dst = C + (size_t)(m0 + t) * N + n0 + r;
-                if (atomic_out) red_add_s32(dst, v);
-                else *dst = v;
+                const size_t idx = (size_t)(m0 + t) * N + n0 + r;
+                if (mult) reinterpret_cast<int8_t *>(C)[idx] = requant_i8(v, mult[n0 + r]);
+                else if (atomic_out) red_add_s32(C + idx, v);
+                else C[idx] = v;
             }
         }
     }
@@ -174,7 +175,7 @@ void launch_one(const Problem &p, int split_k, cudaStream_t stream)
     dim3 grid((p.N + kWarps * R - 1) / (kWarps * R), splits, (p.M + MT - 1) / MT);
     gemv_int_kernel<R, MT, INT2><<<grid, kWarps * 32, 0, stream>>>(
         static_cast<const int8_t *>(p.A), static_cast<const uint8_t *>(p.W),
-        static_cast<int32_t *>(p.C), p.M, p.N, p.K, cps, split_k > 1 ? 1 : 0);
+        static_cast<int32_t *>(p.C), p.M, p.N, p.K, cps, split_k > 1 ? 1 : 0, p.mult);
 }
 
 template <int R, bool INT2>

@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
                int M, int N, int K, int gs, int kb_per_split, int units, int atomic_out,
-               unsigned int *err)
+               const float *__restrict__ mult, unsigned int *err)
 {
     using T = Traits<MODE>;
     using L = Smem<MODE, BN, STAGES>;
@@ -592,6 +592,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             ok = __all_sync(0xffffffffu, ok && !*abort_flag);
             if (!ok) break;
             const int n = w.n0 + r;
+            // int8 requantisation (int32 modes): this lane's output-channel multiplier
+            const float rq = (T::c_bytes == 4 && mult && n < N) ? mult[n] : 0.f;
             const uint32_t lane_addr =
                 tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
 #pragma unroll 1
@@ -619,9 +621,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                             else *dst = __float2half_rn(x);
                         }
                     } else if (n < N) {
-                        int32_t *dst = static_cast<int32_t *>(C) + (size_t)t * N + n;
-                        if (atomic_out) red_add_s32(dst, (int)v[e]);
-                        else *dst = (int)v[e];
+                        const size_t idx = (size_t)t * N + n;
+                        if (mult) static_cast<int8_t *>(C)[idx] = requant_i8((int)v[e], rq);
+                        else if (atomic_out) red_add_s32(static_cast<int32_t *>(C) + idx, (int)v[e]);
+                        else static_cast<int32_t *>(C)[idx] = (int)v[e];
                     }
                 }
             }
@@ -733,7 +736,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     kern<<<grid, kThreads, L::total, stream>>>(
         tw, ta, static_cast<const __half *>(p.scales),
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, p.C, p.M, p.N, p.K, p.gs,
-        kbps, (int)units, split_k > 1 ? 1 : 0, err);
+        kbps, (int)units, split_k > 1 ? 1 : 0, p.mult, err);
     return cudaGetLastError();
 }
 

@@ -179,6 +179,19 @@ qg_status qgemm_w8a8(const int8_t *A, const int8_t *W, int32_t *C, int M, int N,
                      int group_size, int split_k, int has_zero, cudaStream_t stream);
 
 /*
+ * W8A8 with int8 output. A: int8 [M, K]. W: int8 [N, K]. mult: fp32 [N] (one multiplier per
+ * output channel). C: int8 [M, N],
+ *     C[m, n] = clamp(rint(float(acc[m, n]) * mult[n]), -128, 127),   acc = sum_k A[m,k] W[n,k],
+ * acc exact in int32, its conversion to binary32 and the product correctly rounded, rint half to
+ * even. microsoft/BitBLAS issue #252's configuration listing has int8 x int8 configurations
+ * with an int8 output type; the pages do not state the requantisation, this per-channel form
+ * is the reading. The K reduction is never split (the rounding needs the whole sum).
+ * Requires K % 16 == 0; A, W 16-byte aligned, mult 4-byte aligned, C any alignment.
+ */
+qg_status qgemm_w8a8_requant(const int8_t *A, const int8_t *W, const float *mult, int8_t *C,
+                             int M, int N, int K, cudaStream_t stream);
+
+/*
  * W2A8. A: int8 [M, K]. Wq: uint32 [N, K/16], value k of row n is the two's-complement
  * 2-bit field at bits 2*(k%16) of word k/16 (values -2..1). C: int32 [M, N], exact.
  * group_size must be -1 or 0 and has_zero 0. Requires K % 64 == 0.
