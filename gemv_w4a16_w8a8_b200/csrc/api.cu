@@ -196,8 +196,8 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     c.bk = k_per_slab(p.op);
     // packed weights: the deepest ring that still leaves three dequant buffers (measured faster
     // than one more TMA stage with two); other ops: the deepest ring that fits
-    c.stages = tc_max_stages(p.op, c.bn);
-    if ((p.op == QG_OP_W4A16 || p.op == QG_OP_W2A8) && c.stages > 2 && tc_dq_buffers(p.op, c.bn, c.stages) < 3)
+    c.stages = tc_max_stages(p, c.bn);
+    if ((p.op == QG_OP_W4A16 || p.op == QG_OP_W2A8) && c.stages > 2 && tc_dq_buffers(p, c.bn, c.stages) < 3)
         --c.stages;
     c.swap_ab = 1;
     const long tiles = (long)((p.N + 127) / 128) * ((p.M + c.bn - 1) / c.bn);
@@ -449,7 +449,7 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
         const int bns[2] = {base.bn, base.bn / 2};
         for (int bi = 0; bi < 2; ++bi) {
             if (bns[bi] < 16) continue;
-            for (int st = 2; st <= 5; ++st)
+            for (int st : {2, 3, 4, 5, 8, 16})
                 for (int sk = 1; sk <= 8; sk *= 2) {
                     qgemm_config_t t = base;
                     t.bn = bns[bi];

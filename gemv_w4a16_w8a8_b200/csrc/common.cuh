@@ -70,9 +70,9 @@ bool gemv_w2a8_tma_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
 bool tc_supports(const Problem &p, const qgemm_config_t &cfg);
 // Deepest pipeline (2..5) whose shared memory fits for this op and token tile.
-int tc_max_stages(int op, int bn);
+int tc_max_stages(const Problem &p, int bn);
 // Number of upcast-weight buffers the tensor-core kernel keeps for this ring depth (0: none).
-int tc_dq_buffers(int op, int bn, int stages);
+int tc_dq_buffers(const Problem &p, int bn, int stages);
 
 // ------------------------------------------------------------------------------------------
 // PTX wrappers

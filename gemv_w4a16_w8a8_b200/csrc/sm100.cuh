@@ -66,21 +66,29 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Wait for the phase of `bar` with the given parity to complete. Gives up after the time
-// limit (raising the error word and the CTA's abort flag) or when another role gave up. The
-// thread sleeps inside try_wait between checks of the clock and the abort flag.
+// limit (raising the error word and the CTA's abort flag) or when another role gave up. A
+// waiting warp must not take issue slots or pipes from the warps that work: it sleeps inside
+// try_wait, reads the clock and the abort flag only every 64 tries (the clock read goes to a
+// shared pipe), and backs off with nanosleep once the wait runs long.
 __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                        unsigned int *err)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            if (err) atomicOr(err, 1u);
-            return false;
+    uint64_t t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            const uint64_t now = global_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                if (err) atomicOr(err, 1u);
+                return false;
+            }
         }
+        if (i > 256u) __nanosleep(500);
     }
 }
 

@@ -110,29 +110,42 @@ template <int MODE> struct Traits {
 //     STAGES activation slabs (TMA -> MMA), kPackedStages packed weight slabs (TMA -> upcast;
 //     4 KB each, so the upcast can run far ahead) and DQ upcast weight slabs (upcast -> MMA).
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kPackedStages = 12;
 
-constexpr int smem_total(bool packed, int bn, int stages, int dq)
+// Packed weights move PG slabs per copy: PG = 4 reads 128 contiguous bytes of each weight row
+// (HBM serves long row runs far better than 32-byte ones); PG = 1 when K is not a multiple of
+// four slabs. The ring holds kPackedStages copies.
+constexpr int packed_stages(int pg, int bn) { return pg == 1 ? 12 : (bn <= 64 ? 6 : 4); }
+
+constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg)
 {
-    return packed ? 1024 + stages * bn * kSlabBytes + kPackedStages * kRowsW * 32 +
+    return packed ? 1024 + stages * bn * kSlabBytes + packed_stages(pg, bn) * kRowsW * 32 * pg +
                         dq * kRowsW * kSlabBytes +
-                        8 * (2 * stages + 2 * kPackedStages + 2 * dq + 5) + 16
+                        8 * (2 * stages + 2 * packed_stages(pg, bn) + 2 * dq + 5) + 16
                   : 1024 + stages * (kRowsW * kSlabBytes + bn * kSlabBytes) + 8 * (2 * stages + 5) +
                         16;
 }
 
-constexpr int dq_buffers(bool packed, int bn, int stages)
+// Upcast-weight buffers between the dequantisation warps and the MMA: as many as fit, up to 8.
+// Each buffer makes a round trip (upcast, fence, arrive, MMA, commit, release) whose latency
+// bounds the throughput when the token tile is small, so small tiles take the most.
+// The upcast of a packed copy waits for PG free buffers before it hands any over, so the ring
+// holds at least max(2, PG); a plan that cannot is reported as not fitting (smem_bytes).
+constexpr int min_dq(int pg) { return pg < 2 ? 2 : pg; }
+constexpr int dq_buffers(bool packed, int bn, int stages, int pg)
 {
-    return !packed ? 0 : (smem_total(true, bn, stages, 3) <= kMaxSmem ? 3 : 2);
+    if (!packed) return 0;
+    int d = 8;
+    while (d > min_dq(pg) && smem_total(true, bn, stages, d, pg) > kMaxSmem) --d;
+    return d;
 }
 
-template <int MODE, int BN, int STAGES> struct Smem {
+template <int MODE, int BN, int STAGES, int PG> struct Smem {
     static constexpr bool packed = Traits<MODE>::packed;
     static constexpr int a_bytes = BN * kSlabBytes;
     static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
-    static constexpr int pw_bytes = kRowsW * 32;                 // packed weight slab
-    static constexpr int sp = packed ? kPackedStages : 0;
-    static constexpr int dq = dq_buffers(packed, BN, STAGES);
+    static constexpr int pw_bytes = kRowsW * 32 * PG;            // packed weight copy (PG slabs)
+    static constexpr int sp = packed ? packed_stages(PG, BN) : 0;
+    static constexpr int dq = dq_buffers(packed, BN, STAGES, PG);
     static constexpr int dq_bytes = kRowsW * kSlabBytes;
     // byte offsets from the 1024-aligned base
     static constexpr int ring_bytes = packed ? STAGES * a_bytes : STAGES * (w_bytes + a_bytes);
@@ -140,7 +153,7 @@ template <int MODE, int BN, int STAGES> struct Smem {
     static constexpr int dq_off = pw_off + sp * pw_bytes;
     static constexpr int bar_off = dq_off + dq * dq_bytes;
     static constexpr int nbars = 2 * STAGES + 2 * sp + 2 * dq + 5;
-    static constexpr int total = smem_total(packed, BN, STAGES, dq);
+    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG);
 };
 
 // two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
@@ -247,7 +260,7 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
 //   warp 4     TMA producer          warp 5  TMEM allocation + MMA issue
 //   warp 6     TMA producer of packed weight slabs (packed formats)
 //   warps 8-15 dequantisation of packed weights (two threads per weight row of the tile)
-template <int MODE, int BN, int STAGES>
+template <int MODE, int BN, int STAGES, int PG>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
@@ -255,7 +268,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                const float *__restrict__ mult, unsigned int *err)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES>;
+    using L = Smem<MODE, BN, STAGES, PG>;
     constexpr uint32_t kCols = tmem_cols<BN>();
     constexpr uint32_t kIdesc = instr_desc<MODE, BN>();
 
@@ -296,12 +309,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
+        // the 8 dequantisation warps arrive once each (lane 0, after __syncwarp): one arrival
+        // per thread would serialise 256 shared-memory atomics on one barrier every slab
         for (int p = 0; p < SP; ++p) {
             mbar_init(pfull_bar(p), 1);
-            mbar_init(pempty_bar(p), 256);
+            mbar_init(pempty_bar(p), 8);
         }
         for (int d = 0; d < DQ; ++d) {
-            mbar_init(dqf_bar(d), 256);
+            mbar_init(dqf_bar(d), 8);
             mbar_init(dqe_bar(d), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -360,7 +375,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             bool stop = false;
             for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
                 const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
-                for (int i = 0; i < w.nk; ++i, ++it) {
+                // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
+                for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
                     if (!mbar_wait(pempty_bar(p), ((it / SP) & 1) ^ 1, abort_flag, err)) {
                         stop = true;
@@ -387,29 +403,43 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 if (!mbar_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
                 tc_fence_after();
                 const uint32_t dtm = tmem_base + (uint32_t)(b * BN);
-                for (int i = 0; i < w.nk; ++i, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!mbar_wait(full_bar(s), ph, abort_flag, err)) {
+                // MB slabs per pass (the slabs of one packed copy): every wait and fence of this
+                // thread costs far more than issuing an MMA, so they are paid once per pass. The
+                // upcast buffers of a pass are handed over in order by the same warps, so the
+                // last one's barrier covers the others.
+                // (a pass waits for MB activation stages at once, so MB is PG only when the
+                // activation ring holds that many)
+                constexpr int MB = STAGES >= PG ? PG : 1;
+                for (int i = 0; i < w.nk; i += MB, it += MB) {
+                    bool ready = true;
+                    if constexpr (T::packed)
+                        ready = mbar_wait(dqf_bar((it + MB - 1) % DQ), ((it + MB - 1) / DQ) & 1,
+                                          abort_flag, err);
+#pragma unroll
+                    for (int q = 0; q < MB && ready; ++q)
+                        ready = mbar_wait(full_bar((it + q) % STAGES), ((it + q) / STAGES) & 1,
+                                          abort_flag, err);
+                    if (!ready) {
                         stop = true;
                         break;
                     }
-                    const int d = T::packed ? it % DQ : 0;
-                    if constexpr (T::packed) {
-                        if (!mbar_wait(dqf_bar(d), (it / DQ) & 1, abort_flag, err)) {
-                            stop = true;
-                            break;
-                        }
-                    }
                     tc_fence_after();
-                    const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
-                    const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
-                        mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
-                                        (i | k) != 0 ? 1u : 0u);
-                    mma_commit(empty_bar(s));
-                    if constexpr (T::packed) mma_commit(dqe_bar(d));
+                    for (int q = 0; q < MB; ++q) {
+                        const int s = (it + q) % STAGES;
+                        const int d = T::packed ? (it + q) % DQ : 0;
+                        const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
+                        const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
+                            mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                            (i + q | k) != 0 ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int q = 0; q < MB; ++q) {
+                        mma_commit(empty_bar((it + q) % STAGES));
+                        if constexpr (T::packed) mma_commit(dqe_bar((it + q) % DQ));
+                    }
                 }
                 mma_commit(accf_bar(b));
                 ++j;
@@ -534,10 +564,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 ++ahead.i;
                 settle(ahead);
             }
-            int it = 0;
-            while (cur.u < units) {
-                const int p = it % SP, d = it % DQ;
-                uint32_t sc2 = 0u, nz2 = 0u;             // (s, s) and (-z s, -z s) in fp16
+            // scale and zero of the slab at cur as fp16 pairs (s, s) and (-z s, -z s); advances
+            // the scale window or the look-ahead of the per-slab fallback
+            auto slab_scales = [&](uint32_t &sc2, uint32_t &nz2) {
+                sc2 = 0u;
+                nz2 = 0u;
                 if (windowed) {
                     const int g = group_of(cur);
                     if (wcur.u != cur.u || g < wcur.gb || g >= wcur.gb + 8) {
@@ -560,19 +591,60 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     ++ahead.i;
                     settle(ahead);
                 }
-                if (!mbar_wait(pfull_bar(p), (it / SP) & 1, abort_flag, err)) break;
-                const uint32_t *packed = reinterpret_cast<const uint32_t *>(pw_tile(p));
-                const uint4 pk = *reinterpret_cast<const uint4 *>(packed + r * 8 +
+            };
+            // PG slabs (one packed copy) per pass: the PG upcasts are independent, so their
+            // latencies overlap; one proxy fence covers all of them
+            int it = 0;
+            while (cur.u < units) {
+                uint32_t sc2[PG], nz2[PG];
+#pragma unroll
+                for (int j = 0; j < PG; ++j) {
+                    slab_scales(sc2[j], nz2[j]);
+                    if (j + 1 < PG) ++cur.i;   // a copy never straddles units
+                }
+                const int pc = it / PG, pp = pc % SP;
+                // waits decide for the whole warp: the warp-level hand-overs below need all lanes
+                if (!__all_sync(0xffffffffu, mbar_wait(pfull_bar(pp), (pc / SP) & 1, abort_flag, err)))
+                    break;
+                uint4 pk[PG];
+#pragma unroll
+                for (int j = 0; j < PG; ++j) {
+                    if constexpr (PG == 1) {
+                        const uint32_t *packed = reinterpret_cast<const uint32_t *>(pw_tile(pp));
+                        pk[j] = *reinterpret_cast<const uint4 *>(packed + r * 8 +
                                                                  4 * (h ^ ((r >> 2) & 1)));
-                mbar_arrive(pempty_bar(p));          // the packed slot is free once read
-                if (!mbar_wait(dqe_bar(d), ((it / DQ) & 1) ^ 1, abort_flag, err)) break;
-                if constexpr (is_w4(MODE))
-                    dequant_w4<MODE == kW4A16I>(pk, w_dq(d), r, h, sc2, nz2);
-                else
-                    dequant_w2(pk, w_dq(d), r, h);
+                    } else {
+                        // 128-byte rows under the 128-byte swizzle: 16-byte piece c of row r
+                        // sits at c ^ (r & 7); slab j's half h is piece 2 j + h
+                        pk[j] = *reinterpret_cast<const uint4 *>(pw_tile(pp) + r * 128 +
+                                                                 16 * ((2 * j + h) ^ (r & 7)));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty_bar(pp));   // the packed copy is read in full
+                bool ok = true;
+#pragma unroll
+                for (int j = 0; j < PG; ++j) {
+                    const int d = (it + j) % DQ;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(dqe_bar(d), (((it + j) / DQ) & 1) ^ 1, abort_flag, err))) {
+                        ok = false;
+                        break;
+                    }
+                    if constexpr (is_w4(MODE))
+                        dequant_w4<MODE == kW4A16I>(pk[j], w_dq(d), r, h, sc2[j], nz2[j]);
+                    else
+                        dequant_w2(pk[j], w_dq(d), r, h);
+                }
+                if (!ok) break;
+                // every thread's upcast stores become visible to the tensor core (async proxy),
+                // then one arrival per warp hands the buffers over
                 fence_proxy_async_smem();
-                mbar_arrive(dqf_bar(d));
-                ++it;
+                __syncwarp();
+                if (lane == 0)
+#pragma unroll
+                    for (int j = 0; j < PG; ++j) mbar_arrive(dqf_bar((it + j) % DQ));
+                it += PG;
                 ++cur.i;
                 settle(cur);
             }
@@ -658,19 +730,30 @@ int mode_of(int op)
     }
 }
 
-int smem_bytes(int mode, int bn, int stages)
+int smem_bytes(int mode, int bn, int stages, int pg)
 {
     const bool packed = (is_w4(mode) || mode == kW2A8);
-    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages));
+    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg), pg);
 }
 
-template <int MODE, int BN, int STAGES>
+// slabs per packed-weight copy for this problem and tile: 4 when K holds a whole number of
+// 4-slab runs and that plan fits in shared memory, else 1
+int packed_group(const Problem &p, int bn, int stages)
+{
+    const int mode = mode_of(p.op);
+    if (!(is_w4(mode) || mode == kW2A8)) return 1;
+    const int kps = is_w4(mode) ? 64 : 128;
+    if (p.K % kps || (p.K / kps) % 4) return 1;
+    return smem_bytes(mode, bn, stages, 4) <= kMaxSmem ? 4 : 1;
+}
+
+template <int MODE, int BN, int STAGES, int PG>
 cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES>;
+    using L = Smem<MODE, BN, STAGES, PG>;
     if (L::total > kMaxSmem) return cudaErrorInvalidConfiguration;
-    auto kern = tc_gemm_kernel<MODE, BN, STAGES>;
+    auto kern = tc_gemm_kernel<MODE, BN, STAGES, PG>;
     // the dynamic shared-memory opt-in is per device: remember it per device
     static std::mutex mu;
     static bool opted_in[64] = {};
@@ -700,19 +783,19 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                       CU_TENSOR_MAP_SWIZZLE_128B);
     } else if constexpr (is_w4(MODE)) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
-                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_32B) &&
+                      8 * PG, kRowsW, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
                       BN, CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 16, p.N, (uint64_t)p.K / 4,
-                      8, kRowsW, CU_TENSOR_MAP_SWIZZLE_32B) &&
+                      8 * PG, kRowsW, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (!ok) return cudaErrorInvalidValue;
 
     const int nkb = (p.K + T::k_per_slab - 1) / T::k_per_slab;
-    const int kbps = (nkb + split_k - 1) / split_k;
+    const int kbps = ((nkb + split_k - 1) / split_k + PG - 1) / PG * PG;   // whole copies
     const int splits = (nkb + kbps - 1) / kbps;
     const int n_tiles = (p.N + kRowsW - 1) / kRowsW;
     const int t_tiles = (p.M + BN - 1) / BN;
@@ -740,17 +823,33 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     return cudaGetLastError();
 }
 
+template <int MODE, int BN, int PG>
+cudaError_t launch_stages_pg(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                             cudaStream_t stream)
+{
+    switch (c.stages) {
+    case 2: return launch_t<MODE, BN, 2, PG>(p, c.split_k, err, stream);
+    case 3: return launch_t<MODE, BN, 3, PG>(p, c.split_k, err, stream);
+    case 4: return launch_t<MODE, BN, 4, PG>(p, c.split_k, err, stream);
+    case 5: return launch_t<MODE, BN, 5, PG>(p, c.split_k, err, stream);
+    default: break;
+    }
+    // deep activation rings for small token tiles: a small activation copy waits ~2-3 us behind
+    // the weight stream, so only many stages in flight keep the MMA fed
+    if constexpr (BN <= 64) {
+        if (c.stages == 8) return launch_t<MODE, BN, 8, PG>(p, c.split_k, err, stream);
+        if (c.stages == 16) return launch_t<MODE, BN, 16, PG>(p, c.split_k, err, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
 template <int MODE, int BN>
 cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                           cudaStream_t stream)
 {
-    switch (c.stages) {
-    case 2: return launch_t<MODE, BN, 2>(p, c.split_k, err, stream);
-    case 3: return launch_t<MODE, BN, 3>(p, c.split_k, err, stream);
-    case 4: return launch_t<MODE, BN, 4>(p, c.split_k, err, stream);
-    case 5: return launch_t<MODE, BN, 5>(p, c.split_k, err, stream);
-    default: return cudaErrorInvalidValue;
-    }
+    if constexpr (is_w4(MODE) || MODE == kW2A8)
+        if (packed_group(p, BN, c.stages) == 4) return launch_stages_pg<MODE, BN, 4>(p, c, err, stream);
+    return launch_stages_pg<MODE, BN, 1>(p, c, err, stream);
 }
 
 template <int MODE>
@@ -773,9 +872,11 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
 {
     if (c.path != QG_PATH_TC) return false;
     if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
-    if (c.stages < 2 || c.stages > 5) return false;
+    if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 64 && (c.stages == 8 || c.stages == 16))))
+        return false;
     if (c.split_k < 1 || c.split_k > 64) return false;
-    if (smem_bytes(mode_of(p.op), c.bn, c.stages) > kMaxSmem) return false;
+    if (smem_bytes(mode_of(p.op), c.bn, c.stages, packed_group(p, c.bn, c.stages)) > kMaxSmem)
+        return false;
     if (p.op == QG_OP_W4A16 && (p.K % 32 || p.gs % 32 || p.K % p.gs)) return false;
     if (p.op == QG_OP_W2A8 && p.K % 64) return false;
     if (p.op == QG_OP_W8A8 && p.K % 16) return false;
@@ -783,17 +884,27 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
     return true;
 }
 
-int tc_dq_buffers(int op, int bn, int stages)
+int tc_dq_buffers(const Problem &p, int bn, int stages)
 {
-    const int mode = mode_of(op);
-    return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages);
+    const int mode = mode_of(p.op);
+    return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages, packed_group(p, bn, stages));
 }
 
-int tc_max_stages(int op, int bn)
+// the deepest activation ring (2..5, or 16 / 8 for token tiles up to 64) that keeps the grouped
+// packed copies when K allows them
+int tc_max_stages(const Problem &p, int bn)
 {
-    int s = 5;
-    while (s > 2 && smem_bytes(mode_of(op), bn, s) > kMaxSmem) --s;
-    return s;
+    const int mode = mode_of(p.op);
+    // grouped packed copies first (measured faster than one more activation stage without)
+    const bool groupable = packed_group(p, bn, 2) == 4;
+    for (int pg : {4, 1}) {
+        if (pg == 4 && !groupable) continue;
+        for (int s : {16, 8, 5, 4, 3, 2}) {
+            if (s > 5 && bn > 64) continue;
+            if (smem_bytes(mode, bn, s, pg) <= kMaxSmem) return s;
+        }
+    }
+    return 2;
 }
 
 cudaError_t launch_tc(const Problem &p, const qgemm_config_t &c, unsigned int *err,

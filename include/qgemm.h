@@ -90,7 +90,7 @@ typedef struct qgemm_config_t {
     int32_t bm;      /* TC: tile extent along M                                              */
     int32_t bn;      /* TC: tile extent along N                                              */
     int32_t bk;      /* TC: tile extent along K                                              */
-    int32_t stages;  /* TC: depth of the shared-memory pipeline (2..5)                       */
+    int32_t stages;  /* TC: activation ring depth (2..5; also 8, 16 for bn <= 64)           */
     int32_t split_k; /* number of K parts (1 = no atomics)                                   */
     int32_t swap_ab; /* TC: 1 = weights fill the MMA's M side, tokens its N side             */
 } qgemm_config_t;
