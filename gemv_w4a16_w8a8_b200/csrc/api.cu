@@ -194,11 +194,21 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     c.bm = 128;
     c.bn = pow2_at_least(p.M, 16, 256);
     c.bk = k_per_slab(p.op);
-    // packed weights: the deepest ring that still leaves three dequant buffers (measured faster
-    // than one more TMA stage with two); other ops: the deepest ring that fits
+    // packed weights: the deepest ring that still leaves three dequant buffers (four for token
+    // tiles of 128 and more, which hand them over slab by slab; both measured faster than a
+    // deeper activation ring with fewer); other ops: the deepest ring that fits
     c.stages = tc_max_stages(p, c.bn);
-    if ((p.op == QG_OP_W4A16 || p.op == QG_OP_W2A8) && c.stages > 2 && tc_dq_buffers(p, c.bn, c.stages) < 3)
-        --c.stages;
+    if (p.op == QG_OP_W4A16 || p.op == QG_OP_W2A8) {
+        const int want = c.bn >= 128 ? 4 : 3;
+        for (int st : {16, 8, 5, 4, 3, 2}) {
+            if (st > c.stages) continue;
+            qgemm_config_t t = c;
+            t.stages = st;
+            t.split_k = 1;
+            c.stages = st;
+            if (st == 2 || (tc_supports(p, t) && tc_dq_buffers(p, c.bn, st) >= want)) break;
+        }
+    }
     c.swap_ab = 1;
     const long tiles = (long)((p.N + 127) / 128) * ((p.M + c.bn - 1) / c.bn);
     const long nkb = (p.K + c.bk - 1) / c.bk;

@@ -92,6 +92,15 @@ __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, vol
     }
 }
 
+// The whole warp waits for the phase; every lane returns the same decision (false if any lane
+// gave up). The first test is inline, so a phase that is already complete costs one try_wait.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned int *err)
+{
+    const bool ok = mbar_try_wait(bar, parity) || mbar_wait(bar, parity, abort_flag, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
                                             int x, int y)
 {

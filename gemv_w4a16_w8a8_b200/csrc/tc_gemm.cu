@@ -113,29 +113,50 @@ constexpr int kMaxSmem = 227 * 1024;
 
 // Packed weights move PG slabs per copy: PG = 4 reads 128 contiguous bytes of each weight row
 // (HBM serves long row runs far better than 32-byte ones); PG = 1 when K is not a multiple of
-// four slabs. The ring holds kPackedStages copies.
-constexpr int packed_stages(int pg, int bn) { return pg == 1 ? 12 : (bn <= 64 ? 6 : 4); }
+// four slabs.
+//
+// Upcast weight buffers go from the dequantisation warps to the MMA either one slab at a time
+// (token tiles of 128 and more: an MMA slab is long enough to hide a hand-over, and the MMA must
+// not wait for a whole copy) or one packed copy at a time (smaller tiles: there the hand-overs
+// themselves are the cost, and one proxy fence and one arrival per copy are paid instead of PG).
+constexpr bool per_slab_handoff(int bn) { return bn >= 128; }
+// one word per dequantisation thread (see the release of a packed copy)
+constexpr int kSinkBytes = 256 * 4;
+// the fewest upcast buffers a plan may have, and how many it should keep before the packed ring
+// gives up copies for them
+constexpr int min_dq(int pg, int bn) { return (pg < 2 || per_slab_handoff(bn)) ? 2 : pg; }
+constexpr int want_dq(int pg, int bn) { return per_slab_handoff(bn) ? 3 : min_dq(pg, bn); }
 
-constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg)
+constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg, int sp)
 {
-    return packed ? 1024 + stages * bn * kSlabBytes + packed_stages(pg, bn) * kRowsW * 32 * pg +
-                        dq * kRowsW * kSlabBytes +
-                        8 * (2 * stages + 2 * packed_stages(pg, bn) + 2 * dq + 5) + 16
+    return packed ? 1024 + stages * bn * kSlabBytes + sp * kRowsW * 32 * pg +
+                        dq * kRowsW * kSlabBytes + kSinkBytes + 8 * (2 * stages + 2 * sp + 2 * dq + 5) +
+                        16
                   : 1024 + stages * (kRowsW * kSlabBytes + bn * kSlabBytes) + 8 * (2 * stages + 5) +
                         16;
 }
 
-// Upcast-weight buffers between the dequantisation warps and the MMA: as many as fit, up to 8.
-// Each buffer makes a round trip (upcast, fence, arrive, MMA, commit, release) whose latency
-// bounds the throughput when the token tile is small, so small tiles take the most.
-// The upcast of a packed copy waits for PG free buffers before it hands any over, so the ring
-// holds at least max(2, PG); a plan that cannot is reported as not fitting (smem_bytes).
-constexpr int min_dq(int pg) { return pg < 2 ? 2 : pg; }
+// Packed-weight copies in flight: 12 single slabs, or 6 / 4 grouped copies; for token tiles of
+// 128 and more, fewer when a deep activation ring would otherwise leave less than want_dq upcast
+// buffers (one grouped copy holds 4 slabs, so 2-3 copies already run far ahead of the MMA).
+constexpr int packed_stages(int pg, int bn, int stages)
+{
+    if (pg == 1) return 12;
+    if (bn <= 64) return 6;
+    int sp = 4;
+    while (sp > 2 && smem_total(true, bn, stages, want_dq(pg, bn), pg, sp) > kMaxSmem) --sp;
+    return sp;
+}
+
+// Upcast-weight buffers: as many as fit, up to 8. Each buffer makes a round trip (upcast, fence,
+// arrive, MMA, commit, release) whose latency bounds the throughput when the token tile is small,
+// so small tiles take the most. A plan below min_dq is reported as not fitting (smem_bytes).
 constexpr int dq_buffers(bool packed, int bn, int stages, int pg)
 {
     if (!packed) return 0;
+    const int sp = packed_stages(pg, bn, stages);
     int d = 8;
-    while (d > min_dq(pg) && smem_total(true, bn, stages, d, pg) > kMaxSmem) --d;
+    while (d > min_dq(pg, bn) && smem_total(true, bn, stages, d, pg, sp) > kMaxSmem) --d;
     return d;
 }
 
@@ -144,16 +165,17 @@ template <int MODE, int BN, int STAGES, int PG> struct Smem {
     static constexpr int a_bytes = BN * kSlabBytes;
     static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
     static constexpr int pw_bytes = kRowsW * 32 * PG;            // packed weight copy (PG slabs)
-    static constexpr int sp = packed ? packed_stages(PG, BN) : 0;
+    static constexpr int sp = packed ? packed_stages(PG, BN, STAGES) : 0;
     static constexpr int dq = dq_buffers(packed, BN, STAGES, PG);
     static constexpr int dq_bytes = kRowsW * kSlabBytes;
     // byte offsets from the 1024-aligned base
     static constexpr int ring_bytes = packed ? STAGES * a_bytes : STAGES * (w_bytes + a_bytes);
     static constexpr int pw_off = ring_bytes;
     static constexpr int dq_off = pw_off + sp * pw_bytes;
-    static constexpr int bar_off = dq_off + dq * dq_bytes;
+    static constexpr int sink_off = dq_off + dq * dq_bytes;
+    static constexpr int bar_off = sink_off + (packed ? kSinkBytes : 0);
     static constexpr int nbars = 2 * STAGES + 2 * sp + 2 * dq + 5;
-    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG);
+    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG, sp);
 };
 
 // two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
@@ -340,36 +362,41 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
+    // The producer and MMA warps run their loops with all 32 lanes, so that control flow, slot
+    // indices, coordinates and descriptors stay warp-uniform: the compiler then keeps them in
+    // uniform registers, which is where TMA and tcgen05.mma take their operands from (computed
+    // in a one-lane branch they must be moved there first, which costs more than the issue
+    // itself). Lane 0 issues; every lane waits, and the warp takes one decision per wait.
     if (warp == 4) {
-        if (lane == 0) {
-            // ---------------- TMA producer (weight + activation slabs, or activations) --------
-            constexpr uint32_t kTx = L::packed ? L::a_bytes : L::w_bytes + L::a_bytes;
-            int it = 0;
-            bool stop = false;
-            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
-                for (int i = 0; i < w.nk; ++i, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
-                        stop = true;
-                        break;
-                    }
-                    mbar_expect_tx(full_bar(s), kTx);
-                    const int kb = w.kb0 + i;
-                    if constexpr (!L::packed)
-                        tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kb * T::k_per_slab,
-                                    w.n0);
-                    tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kb * T::k_per_slab, w.t0);
+        // ---------------- TMA producer (weight + activation slabs, or activations) --------
+        constexpr uint32_t kTx = L::packed ? L::a_bytes : L::w_bytes + L::a_bytes;
+        int it = 0;
+        bool stop = false;
+        for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            for (int i = 0; i < w.nk; ++i, ++it) {
+                const int s = it % STAGES;
+                if (!warp_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
+                    stop = true;
+                    break;
                 }
-            }
-            // every copy this thread started must land before the CTA can exit
-            for (int i = max(0, it - STAGES); i < it; ++i) {
-                int dummy_abort = 0;
-                mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+                const int kx = (w.kb0 + i) * T::k_per_slab;
+                if (lane == 0) {
+                    mbar_expect_tx(full_bar(s), kTx);
+                    if constexpr (!L::packed)
+                        tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kx, w.n0);
+                    tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kx, w.t0);
+                }
+                __syncwarp();
             }
         }
+        // every copy this warp started must land before the CTA can exit
+        for (int i = max(0, it - STAGES); i < it; ++i) {
+            int dummy_abort = 0;
+            mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+        }
     } else if (warp == 6) {
-        if (L::packed && lane == 0) {
+        if constexpr (L::packed) {
             // ---------------- TMA producer (packed weight slabs) ----------------
             int it = 0;
             bool stop = false;
@@ -378,12 +405,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
                 for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
-                    if (!mbar_wait(pempty_bar(p), ((it / SP) & 1) ^ 1, abort_flag, err)) {
+                    if (!warp_wait(pempty_bar(p), ((it / SP) & 1) ^ 1, abort_flag, err)) {
                         stop = true;
                         break;
                     }
-                    mbar_expect_tx(pfull_bar(p), L::pw_bytes);
-                    tma_load_2d(smem_u32(pw_tile(p)), &tm_w, pfull_bar(p), (w.kb0 + i) * 8, w.n0);
+                    if (lane == 0) {
+                        mbar_expect_tx(pfull_bar(p), L::pw_bytes);
+                        tma_load_2d(smem_u32(pw_tile(p)), &tm_w, pfull_bar(p), (w.kb0 + i) * 8,
+                                    w.n0);
+                    }
+                    __syncwarp();
                 }
             }
             for (int i = max(0, it - SP); i < it; ++i) {
@@ -392,63 +423,54 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             }
         }
     } else if (warp == 5) {
-        if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            int it = 0, j = 0;
-            bool stop = false;
-            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
-                if (w.nk == 0) continue;
-                const int b = j & 1;
-                if (!mbar_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
-                tc_fence_after();
-                const uint32_t dtm = tmem_base + (uint32_t)(b * BN);
-                // MB slabs per pass (the slabs of one packed copy): every wait and fence of this
-                // thread costs far more than issuing an MMA, so they are paid once per pass. The
-                // upcast buffers of a pass are handed over in order by the same warps, so the
-                // last one's barrier covers the others.
-                // (a pass waits for MB activation stages at once, so MB is PG only when the
-                // activation ring holds that many)
-                constexpr int MB = STAGES >= PG ? PG : 1;
-                for (int i = 0; i < w.nk; i += MB, it += MB) {
-                    bool ready = true;
-                    if constexpr (T::packed)
-                        ready = mbar_wait(dqf_bar((it + MB - 1) % DQ), ((it + MB - 1) / DQ) & 1,
-                                          abort_flag, err);
-#pragma unroll
-                    for (int q = 0; q < MB && ready; ++q)
-                        ready = mbar_wait(full_bar((it + q) % STAGES), ((it + q) / STAGES) & 1,
-                                          abort_flag, err);
-                    if (!ready) {
-                        stop = true;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int q = 0; q < MB; ++q) {
-                        const int s = (it + q) % STAGES;
-                        const int d = T::packed ? (it + q) % DQ : 0;
-                        const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
-                        const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
-                            mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
-                                            (i + q | k) != 0 ? 1u : 0u);
-                    }
-#pragma unroll
-                    for (int q = 0; q < MB; ++q) {
-                        mma_commit(empty_bar((it + q) % STAGES));
-                        if constexpr (T::packed) mma_commit(dqe_bar((it + q) % DQ));
-                    }
+        // ---------------- MMA issuer ----------------
+        // Lane 0 issues the MMAs and the commits: a commit tracks the MMAs its own thread issued.
+        int it = 0, j = 0;
+        bool stop = false;
+        for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            if (w.nk == 0) continue;
+            const int b = j & 1;
+            if (!warp_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
+            tc_fence_after();
+            const uint32_t dtm = tmem_base + (uint32_t)(b * BN);
+            // one slab at a time: wait for its activation stage (and upcast weights), issue its 4
+            // MMAs, then commit its buffers back at once, so that every buffer returns to its
+            // producer as soon as the tensor core is done with it (a commit tracks all MMAs this
+            // thread issued before it)
+            for (int i = 0; i < w.nk; ++i, ++it) {
+                const int s = it % STAGES;
+                const int d = T::packed ? it % DQ : 0;
+                bool ready = true;
+                if constexpr (T::packed) ready = warp_wait(dqf_bar(d), (it / DQ) & 1, abort_flag, err);
+                ready = ready && warp_wait(full_bar(s), (it / STAGES) & 1, abort_flag, err);
+                if (!ready) {
+                    stop = true;
+                    break;
                 }
-                mma_commit(accf_bar(b));
-                ++j;
+                tc_fence_after();
+                const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
+                const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
+                if (lane == 0) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
+                        mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                        (i | k) != 0 ? 1u : 0u);
+                    mma_commit(empty_bar(s));
+                    if constexpr (T::packed) mma_commit(dqe_bar(d));
+                }
+                __syncwarp();
             }
-            // nothing may still run on the tensor cores when TMEM is released
-            mma_commit(final_bar);
-            int dummy_abort = 0;
-            mbar_wait(final_bar, 0, &dummy_abort, nullptr);
+            if (stop) break;
+            if (lane == 0) mma_commit(accf_bar(b));
+            __syncwarp();
+            ++j;
         }
+        // nothing may still run on the tensor cores when TMEM is released
+        if (lane == 0) mma_commit(final_bar);
+        __syncwarp();
+        int dummy_abort = 0;
+        mbar_wait(final_bar, 0, &dummy_abort, nullptr);
     } else if (warp >= 8) {
         // ---------------- dequantisation (packed weights) ----------------
         // 256 threads: thread (h, r) upcasts words 4h..4h+3 of weight row r of every slab. The
@@ -456,6 +478,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         if constexpr (T::packed) {
             const int dq = tid - 256;
             const int r = dq & 127, h = dq >> 7;
+            volatile uint32_t *sink = reinterpret_cast<volatile uint32_t *>(base + L::sink_off);
             const int G = K / gs;
             // cursor over this CTA's slabs: unit u (position i inside it, w its coordinates)
             struct Cursor {
@@ -604,8 +627,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 }
                 const int pc = it / PG, pp = pc % SP;
                 // waits decide for the whole warp: the warp-level hand-overs below need all lanes
-                if (!__all_sync(0xffffffffu, mbar_wait(pfull_bar(pp), (pc / SP) & 1, abort_flag, err)))
-                    break;
+                if (!warp_wait(pfull_bar(pp), (pc / SP) & 1, abort_flag, err)) break;
                 uint4 pk[PG];
 #pragma unroll
                 for (int j = 0; j < PG; ++j) {
@@ -620,14 +642,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                                                                  16 * ((2 * j + h) ^ (r & 7)));
                     }
                 }
+                // The slot goes back to the TMA producer only once every lane's loads of it have
+                // returned: an arrival does not wait for loads still in flight in other lanes, and
+                // the next copy into the slot would overwrite data not yet read. A store of a
+                // value computed from all four loads cannot issue before they return, and the
+                // arrival (a release) is ordered after it.
+                uint32_t landed = 0;
+#pragma unroll
+                for (int j = 0; j < PG; ++j) landed ^= pk[j].x ^ pk[j].y ^ pk[j].z ^ pk[j].w;
+                sink[dq] = landed;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(pempty_bar(pp));   // the packed copy is read in full
                 bool ok = true;
 #pragma unroll
                 for (int j = 0; j < PG; ++j) {
                     const int d = (it + j) % DQ;
-                    if (!__all_sync(0xffffffffu,
-                                    mbar_wait(dqe_bar(d), (((it + j) / DQ) & 1) ^ 1, abort_flag, err))) {
+                    if (!warp_wait(dqe_bar(d), (((it + j) / DQ) & 1) ^ 1, abort_flag, err)) {
                         ok = false;
                         break;
                     }
@@ -635,15 +665,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         dequant_w4<MODE == kW4A16I>(pk[j], w_dq(d), r, h, sc2[j], nz2[j]);
                     else
                         dequant_w2(pk[j], w_dq(d), r, h);
+                    if constexpr (per_slab_handoff(BN)) {
+                        // this slab's upcast stores become visible to the tensor core (async
+                        // proxy), then one arrival per warp hands the buffer over
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(dqf_bar(d));
+                    }
                 }
                 if (!ok) break;
-                // every thread's upcast stores become visible to the tensor core (async proxy),
-                // then one arrival per warp hands the buffers over
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0)
+                if constexpr (!per_slab_handoff(BN)) {
+                    // the same for the whole copy: one fence, then the PG buffers in order
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0)
 #pragma unroll
-                    for (int j = 0; j < PG; ++j) mbar_arrive(dqf_bar((it + j) % DQ));
+                        for (int j = 0; j < PG; ++j) mbar_arrive(dqf_bar((it + j) % DQ));
+                }
                 it += PG;
                 ++cur.i;
                 settle(cur);
@@ -733,7 +771,8 @@ int mode_of(int op)
 int smem_bytes(int mode, int bn, int stages, int pg)
 {
     const bool packed = (is_w4(mode) || mode == kW2A8);
-    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg), pg);
+    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg), pg,
+                      packed ? packed_stages(pg, bn, stages) : 0);
 }
 
 // slabs per packed-weight copy for this problem and tile: 4 when K holds a whole number of
@@ -836,10 +875,10 @@ cudaError_t launch_stages_pg(const Problem &p, const qgemm_config_t &c, unsigned
     }
     // deep activation rings for small token tiles: a small activation copy waits ~2-3 us behind
     // the weight stream, so only many stages in flight keep the MMA fed
-    if constexpr (BN <= 64) {
+    if constexpr (BN <= 128)
         if (c.stages == 8) return launch_t<MODE, BN, 8, PG>(p, c.split_k, err, stream);
+    if constexpr (BN <= 64)
         if (c.stages == 16) return launch_t<MODE, BN, 16, PG>(p, c.split_k, err, stream);
-    }
     return cudaErrorInvalidValue;
 }
 
@@ -872,7 +911,8 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
 {
     if (c.path != QG_PATH_TC) return false;
     if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
-    if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 64 && (c.stages == 8 || c.stages == 16))))
+    if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 128 && c.stages == 8) ||
+          (c.bn <= 64 && c.stages == 16)))
         return false;
     if (c.split_k < 1 || c.split_k > 64) return false;
     if (smem_bytes(mode_of(p.op), c.bn, c.stages, packed_group(p, c.bn, c.stages)) > kMaxSmem)
@@ -890,7 +930,7 @@ int tc_dq_buffers(const Problem &p, int bn, int stages)
     return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages, packed_group(p, bn, stages));
 }
 
-// the deepest activation ring (2..5, or 16 / 8 for token tiles up to 64) that keeps the grouped
+// the deepest activation ring (2..5; 8 for token tiles up to 128, 16 up to 64) that keeps the grouped
 // packed copies when K allows them
 int tc_max_stages(const Problem &p, int bn)
 {
@@ -900,7 +940,7 @@ int tc_max_stages(const Problem &p, int bn)
     for (int pg : {4, 1}) {
         if (pg == 4 && !groupable) continue;
         for (int s : {16, 8, 5, 4, 3, 2}) {
-            if (s > 5 && bn > 64) continue;
+            if ((s == 16 && bn > 64) || (s == 8 && bn > 128)) continue;
             if (smem_bytes(mode, bn, s, pg) <= kMaxSmem) return s;
         }
     }

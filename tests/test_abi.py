@@ -209,11 +209,20 @@ def test_tc_split_fills_the_gpu():
 
 
 def test_tc_config_limits():
-    M, N, K = 256, 512, 1024
-    # packed weights at a 256-token tile: 4 activation stages (128 KB) + 12 packed slabs (48 KB)
-    # + 3 upcast buffers (48 KB) fit; a fifth activation stage does not
+    M, N = 256, 512
+    # K = 1152 (18 slabs, single-slab packed copies) at a 256-token tile: 4 activation stages
+    # (128 KB) + 12 packed slabs (48 KB) + 3 upcast buffers (48 KB) fit; a fifth stage does not
+    K = 1152
     qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 4))
-    for bad in (_tc(256, 5), _tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 5))
+    # K = 1024 (four-slab copies): two grouped copies and two upcast buffers leave room for a
+    # fifth activation stage; 8 stages are for token tiles up to 128, 16 up to 64
+    K = 1024
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 4))
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(256, 5))
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, _tc(128, 8))
+    for bad in (_tc(256, 8), _tc(128, 16), _tc(48, 3), _tc(64, 1), _tc(64, 6), _tc(64, 3, 65)):
         with pytest.raises(qg.QGemmError):
             qg.qgemm_set_config(qg.OP_W4A16, M, N, K, 128, 1, bad)
     qg.qgemm_set_config(qg.OP_DENSE_F16, M, N, K, -1, 0, _tc(256, 4))
