@@ -218,6 +218,42 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     return c;
 }
 
+// Token-major tensor-core tile for few tokens (W4A16): 128 tokens x 256 weight rows per tile, the
+// deepest activation ring that keeps three upcast buffers, and the K split that gives the
+// shortest persistent schedule: whole waves of units, each a run of 4-slab copies, plus a cost
+// per unit for its epilogue, which grows with the tokens it adds into C (fp16 atomics).
+qgemm_config_t tc_toka_default(const Problem &p, int sms)
+{
+    qgemm_config_t c;
+    std::memset(&c, 0, sizeof(c));
+    c.path = QG_PATH_TC;
+    c.bm = 128;
+    c.bn = 256;
+    c.bk = 64;
+    c.swap_ab = 0;
+    c.split_k = 1;
+    for (int st : {4, 3, 2}) {
+        c.stages = st;
+        if (tc_supports(p, c)) break;
+    }
+    const long tiles = (long)((p.N + 255) / 256) * ((p.M + 127) / 128);
+    const int nkb = p.K / 64;
+    double best = 1e30;
+    for (int sk = 1; sk <= 16; ++sk) {
+        const int kbps = ((nkb + sk - 1) / sk + 3) / 4 * 4;
+        const int parts = (nkb + kbps - 1) / kbps;
+        if (parts != sk) continue;   // another split gives the same parts
+        const long units = tiles * parts;
+        const double epi = 2.0 + (parts > 1 ? std::min(p.M, 128) / 8.0 : 0.0);
+        const double cost = (double)((units + sms - 1) / sms) * (kbps + epi);
+        if (cost < best) {
+            best = cost;
+            c.split_k = sk;
+        }
+    }
+    return c;
+}
+
 // Persistent stream-K W4A16 kernel: 64-row x 512-K stages (256 contiguous bytes of each weight
 // row a copy) consumed by 4 row warps x 2 K warps, in the deepest ring shared memory holds (up
 // to 16 stages: HBM needs ~100 KB in flight per SM), one CTA per SM.
@@ -249,6 +285,11 @@ qgemm_config_t heuristic(const Problem &p, int sms, bool allow_stream)
     if (allow_stream && p.op == QG_OP_W4A16 && p.M > 8 && p.M <= 16) {
         qgemm_config_t st = stream_default(p);
         if (gemv_w4a16_stream_supports(p, st)) return st;
+    }
+    // token-major tensor-core tiles up to one tile of tokens (W4A16; groups of whole slabs)
+    if (p.op == QG_OP_W4A16 && p.M > 16 && p.M <= 128) {
+        qgemm_config_t tk = tc_toka_default(p, sms);
+        if (tc_supports(p, tk)) return tk;
     }
     // tensor-core GEMM once there are enough tokens to fill its tile
     if (p.op == QG_OP_DENSE_F16 || p.M > 16) {
@@ -453,6 +494,21 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                         out.push_back(t);
                     }
                 }
+    }
+    if (p.op == QG_OP_W4A16 && p.M <= 256) {
+        qgemm_config_t t = tc_toka_default(p, kDefaultSms);
+        const int best_split = t.split_k;
+        for (int st : {2, 3, 4})
+            for (int sk : {1, 2, 3, 4, 6, 8, 12, 16}) {
+                t.stages = st;
+                t.split_k = sk;
+                if (tc_supports(p, t)) out.push_back(t);
+            }
+        t.split_k = best_split;
+        for (int st : {2, 3, 4}) {
+            t.stages = st;
+            if (tc_supports(p, t)) out.push_back(t);
+        }
     }
     if (p.op == QG_OP_DENSE_F16 || p.M > 1) {
         const qgemm_config_t base = tc_default(p, kDefaultSms);

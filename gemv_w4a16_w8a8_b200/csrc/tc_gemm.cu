@@ -36,6 +36,13 @@ constexpr bool is_w4(int m) { return m == kW4A16 || m == kW4A16I; }
 
 constexpr int kThreads = 512;
 constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
+// Token-major variant (TOKA) for few tokens: the tokens are the MMA's A operand (M = 128; rows
+// past the last token read as zero) and 256 upcast weight rows its B operand (N = 256). An MMA
+// from shared memory costs the same ~100 cycles for any N up to 128 and reaches the full rate
+// only at N = 256, so few tokens in N waste most of the tensor core; in M they do not.
+constexpr int kRowsT = 256;            // weight rows per tile of the token-major variant
+constexpr int kTokT = 128;             // tokens per tile of the token-major variant
+template <bool TOKA> constexpr int wrows() { return TOKA ? kRowsT : kRowsW; }
 constexpr int kSlabBytes = 128;        // bytes of K per stage and row (64 fp16 / 128 int8)
 constexpr int kGroupT = 8;             // token tiles per raster group
 
@@ -127,11 +134,10 @@ constexpr int kSinkBytes = 256 * 4;
 constexpr int min_dq(int pg, int bn) { return (pg < 2 || per_slab_handoff(bn)) ? 2 : pg; }
 constexpr int want_dq(int pg, int bn) { return per_slab_handoff(bn) ? 3 : min_dq(pg, bn); }
 
-constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg, int sp)
+constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg, int sp, int wr = kRowsW)
 {
-    return packed ? 1024 + stages * bn * kSlabBytes + sp * kRowsW * 32 * pg +
-                        dq * kRowsW * kSlabBytes + kSinkBytes + 8 * (2 * stages + 2 * sp + 2 * dq + 5) +
-                        16
+    return packed ? 1024 + stages * bn * kSlabBytes + sp * wr * 32 * pg + dq * wr * kSlabBytes +
+                        kSinkBytes + 8 * (2 * stages + 2 * sp + 2 * dq + 5) + 16
                   : 1024 + stages * (kRowsW * kSlabBytes + bn * kSlabBytes) + 8 * (2 * stages + 5) +
                         16;
 }
@@ -139,35 +145,37 @@ constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg, int sp
 // Packed-weight copies in flight: 12 single slabs, or 6 / 4 grouped copies; for token tiles of
 // 128 and more, fewer when a deep activation ring would otherwise leave less than want_dq upcast
 // buffers (one grouped copy holds 4 slabs, so 2-3 copies already run far ahead of the MMA).
-constexpr int packed_stages(int pg, int bn, int stages)
+constexpr int packed_stages(int pg, int bn, int stages, int wr = kRowsW)
 {
     if (pg == 1) return 12;
     if (bn <= 64) return 6;
     int sp = 4;
-    while (sp > 2 && smem_total(true, bn, stages, want_dq(pg, bn), pg, sp) > kMaxSmem) --sp;
+    while (sp > 2 && smem_total(true, bn, stages, want_dq(pg, bn), pg, sp, wr) > kMaxSmem) --sp;
     return sp;
 }
 
 // Upcast-weight buffers: as many as fit, up to 8. Each buffer makes a round trip (upcast, fence,
 // arrive, MMA, commit, release) whose latency bounds the throughput when the token tile is small,
 // so small tiles take the most. A plan below min_dq is reported as not fitting (smem_bytes).
-constexpr int dq_buffers(bool packed, int bn, int stages, int pg)
+constexpr int dq_buffers(bool packed, int bn, int stages, int pg, int wr = kRowsW)
 {
     if (!packed) return 0;
-    const int sp = packed_stages(pg, bn, stages);
+    const int sp = packed_stages(pg, bn, stages, wr);
     int d = 8;
-    while (d > min_dq(pg, bn) && smem_total(true, bn, stages, d, pg, sp) > kMaxSmem) --d;
+    while (d > min_dq(pg, bn) && smem_total(true, bn, stages, d, pg, sp, wr) > kMaxSmem) --d;
     return d;
 }
 
-template <int MODE, int BN, int STAGES, int PG> struct Smem {
+// BN: tokens per tile (the MMA's N, or its M in the token-major variant); WR weight rows.
+template <int MODE, int BN, int STAGES, int PG, bool TOKA = false> struct Smem {
     static constexpr bool packed = Traits<MODE>::packed;
+    static constexpr int WR = wrows<TOKA>();
     static constexpr int a_bytes = BN * kSlabBytes;
     static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
-    static constexpr int pw_bytes = kRowsW * 32 * PG;            // packed weight copy (PG slabs)
-    static constexpr int sp = packed ? packed_stages(PG, BN, STAGES) : 0;
-    static constexpr int dq = dq_buffers(packed, BN, STAGES, PG);
-    static constexpr int dq_bytes = kRowsW * kSlabBytes;
+    static constexpr int pw_bytes = WR * 32 * PG;                // packed weight copy (PG slabs)
+    static constexpr int sp = packed ? packed_stages(PG, BN, STAGES, WR) : 0;
+    static constexpr int dq = dq_buffers(packed, BN, STAGES, PG, WR);
+    static constexpr int dq_bytes = WR * kSlabBytes;
     // byte offsets from the 1024-aligned base
     static constexpr int ring_bytes = packed ? STAGES * a_bytes : STAGES * (w_bytes + a_bytes);
     static constexpr int pw_off = ring_bytes;
@@ -175,7 +183,7 @@ template <int MODE, int BN, int STAGES, int PG> struct Smem {
     static constexpr int sink_off = dq_off + dq * dq_bytes;
     static constexpr int bar_off = sink_off + (packed ? kSinkBytes : 0);
     static constexpr int nbars = 2 * STAGES + 2 * sp + 2 * dq + 5;
-    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG, sp);
+    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG, sp, WR);
 };
 
 // two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
@@ -257,7 +265,7 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv, int nkb,
-                                        int kbps)
+                                        int kbps, int wr = kRowsW)
 {
     const int tiles = n_tiles * t_tiles;
     const int split = u / tiles;
@@ -269,7 +277,7 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
     const int within = tile - group * per_group;
     Unit w;
     w.t0 = (first_t + within % gt) * BNv;
-    w.n0 = (within / gt) * kRowsW;
+    w.n0 = (within / gt) * wr;
     w.kb0 = split * kbps;
     w.nk = max(0, min(nkb, w.kb0 + kbps) - w.kb0);
     return w;
@@ -281,8 +289,11 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
 //   warps 0-3  epilogue (warp w reads TMEM lanes 32w..32w+31)
 //   warp 4     TMA producer          warp 5  TMEM allocation + MMA issue
 //   warp 6     TMA producer of packed weight slabs (packed formats)
-//   warps 8-15 dequantisation of packed weights (two threads per weight row of the tile)
-template <int MODE, int BN, int STAGES, int PG>
+//   warps 8-15 dequantisation of packed weights (two threads per weight row of the tile, or one
+//              in the token-major variant)
+// TOKA: token-major variant (W4A16): tiles of kTokT = BN tokens x kRowsT weight rows, tokens in
+// the MMA's M, weights in its N; the accumulator holds one token per TMEM lane.
+template <int MODE, int BN, int STAGES, int PG, bool TOKA>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
@@ -290,9 +301,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                const float *__restrict__ mult, unsigned int *err)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES, PG>;
-    constexpr uint32_t kCols = tmem_cols<BN>();
-    constexpr uint32_t kIdesc = instr_desc<MODE, BN>();
+    using L = Smem<MODE, BN, STAGES, PG, TOKA>;
+    static_assert(!TOKA || (is_w4(MODE) && BN == kTokT), "token-major tiles: W4A16, 128 tokens");
+    constexpr int WR = L::WR;
+    constexpr int NMMA = TOKA ? kRowsT : BN;          // the MMA's N (accumulator columns)
+    constexpr uint32_t kCols = tmem_cols<NMMA>();
+    constexpr uint32_t kIdesc = instr_desc<MODE, NMMA>();
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -304,7 +318,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int n_tiles = (N + kRowsW - 1) / kRowsW;
+    const int n_tiles = (N + WR - 1) / WR;
     const int t_tiles = (M + BN - 1) / BN;
     const int nkb = (K + T::k_per_slab - 1) / T::k_per_slab;
 
@@ -373,7 +387,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         int it = 0;
         bool stop = false;
         for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
             for (int i = 0; i < w.nk; ++i, ++it) {
                 const int s = it % STAGES;
                 if (!warp_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
@@ -401,7 +415,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             int it = 0;
             bool stop = false;
             for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
                 // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
                 for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
@@ -428,12 +442,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         int it = 0, j = 0;
         bool stop = false;
         for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
             if (w.nk == 0) continue;
             const int b = j & 1;
             if (!warp_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
             tc_fence_after();
-            const uint32_t dtm = tmem_base + (uint32_t)(b * BN);
+            const uint32_t dtm = tmem_base + (uint32_t)(b * NMMA);
             // one slab at a time: wait for its activation stage (and upcast weights), issue its 4
             // MMAs, then commit its buffers back at once, so that every buffer returns to its
             // producer as soon as the tensor core is done with it (a commit tracks all MMAs this
@@ -449,8 +463,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     break;
                 }
                 tc_fence_after();
-                const uint64_t adesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
-                const uint64_t bdesc = sw128_desc(smem_u32(a_tile(s)));
+                const uint64_t wdesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
+                const uint64_t tdesc = sw128_desc(smem_u32(a_tile(s)));
+                const uint64_t adesc = TOKA ? tdesc : wdesc, bdesc = TOKA ? wdesc : tdesc;
                 if (lane == 0) {
 #pragma unroll
                     for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
@@ -477,7 +492,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         // scale and zero of the next slab are loaded while the current one is processed.
         if constexpr (T::packed) {
             const int dq = tid - 256;
-            const int r = dq & 127, h = dq >> 7;
+            // thread (h, r) upcasts half h of weight row r; in the token-major variant thread r
+            // upcasts both halves of row r (h = 0 then names the slab's scale group: the group
+            // size is a multiple of 64 there)
+            constexpr int NH = TOKA ? 2 : 1;
+            const int r = TOKA ? dq : (dq & 127), h = TOKA ? 0 : (dq >> 7);
             volatile uint32_t *sink = reinterpret_cast<volatile uint32_t *>(base + L::sink_off);
             const int G = K / gs;
             // cursor over this CTA's slabs: unit u (position i inside it, w its coordinates)
@@ -489,10 +508,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 while (c.u < units && c.i >= c.w.nk) {
                     c.u += gridDim.x;
                     c.i = 0;
-                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
                 }
             };
-            Cursor cur{(int)blockIdx.x, 0, unit_of(blockIdx.x, n_tiles, t_tiles, BN, nkb, kb_per_split)};
+            Cursor cur{(int)blockIdx.x, 0, unit_of(blockIdx.x, n_tiles, t_tiles, BN, nkb, kb_per_split, WR)};
             settle(cur);
             // Scales and zeros. Per slab a thread needs s[n][g] and z[n][g] of its row n. Loading
             // those 2-byte values one slab at a time makes every warp touch 32 rows (32 sectors)
@@ -524,7 +543,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             };
             // the window after wnd in this CTA's walk (same unit, or the next unit's first one)
             auto next_window = [&](Window &out, const Window &wnd) {
-                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
                 const int g_last = min(((w.kb0 + w.nk) * 64 - 1) / gs, G - 1);
                 if (wnd.gb + 8 <= g_last) {
                     load_window(out, wnd.u, w, wnd.gb + 8);
@@ -533,7 +552,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 int u = wnd.u + gridDim.x;
                 Unit nw = w;
                 while (u < units) {
-                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
                     if (nw.nk > 0) break;
                     u += gridDim.x;
                 }
@@ -628,20 +647,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 const int pc = it / PG, pp = pc % SP;
                 // waits decide for the whole warp: the warp-level hand-overs below need all lanes
                 if (!warp_wait(pfull_bar(pp), (pc / SP) & 1, abort_flag, err)) break;
-                uint4 pk[PG];
+                uint4 pk[PG][NH];
 #pragma unroll
-                for (int j = 0; j < PG; ++j) {
-                    if constexpr (PG == 1) {
-                        const uint32_t *packed = reinterpret_cast<const uint32_t *>(pw_tile(pp));
-                        pk[j] = *reinterpret_cast<const uint4 *>(packed + r * 8 +
-                                                                 4 * (h ^ ((r >> 2) & 1)));
-                    } else {
-                        // 128-byte rows under the 128-byte swizzle: 16-byte piece c of row r
-                        // sits at c ^ (r & 7); slab j's half h is piece 2 j + h
-                        pk[j] = *reinterpret_cast<const uint4 *>(pw_tile(pp) + r * 128 +
-                                                                 16 * ((2 * j + h) ^ (r & 7)));
+                for (int j = 0; j < PG; ++j)
+#pragma unroll
+                    for (int x = 0; x < NH; ++x) {
+                        const int hv = TOKA ? x : h;
+                        if constexpr (PG == 1) {
+                            const uint32_t *packed = reinterpret_cast<const uint32_t *>(pw_tile(pp));
+                            pk[j][x] = *reinterpret_cast<const uint4 *>(packed + r * 8 +
+                                                                        4 * (hv ^ ((r >> 2) & 1)));
+                        } else {
+                            // 128-byte rows under the 128-byte swizzle: 16-byte piece c of row r
+                            // sits at c ^ (r & 7); slab j's half h is piece 2 j + h
+                            pk[j][x] = *reinterpret_cast<const uint4 *>(
+                                pw_tile(pp) + r * 128 + 16 * ((2 * j + hv) ^ (r & 7)));
+                        }
                     }
-                }
                 // The slot goes back to the TMA producer only once every lane's loads of it have
                 // returned: an arrival does not wait for loads still in flight in other lanes, and
                 // the next copy into the slot would overwrite data not yet read. A store of a
@@ -649,7 +671,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 // arrival (a release) is ordered after it.
                 uint32_t landed = 0;
 #pragma unroll
-                for (int j = 0; j < PG; ++j) landed ^= pk[j].x ^ pk[j].y ^ pk[j].z ^ pk[j].w;
+                for (int j = 0; j < PG; ++j)
+#pragma unroll
+                    for (int x = 0; x < NH; ++x)
+                        landed ^= pk[j][x].x ^ pk[j][x].y ^ pk[j][x].z ^ pk[j][x].w;
                 sink[dq] = landed;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(pempty_bar(pp));   // the packed copy is read in full
@@ -661,10 +686,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         ok = false;
                         break;
                     }
-                    if constexpr (is_w4(MODE))
-                        dequant_w4<MODE == kW4A16I>(pk[j], w_dq(d), r, h, sc2[j], nz2[j]);
-                    else
-                        dequant_w2(pk[j], w_dq(d), r, h);
+#pragma unroll
+                    for (int x = 0; x < NH; ++x) {
+                        if constexpr (is_w4(MODE))
+                            dequant_w4<MODE == kW4A16I>(pk[j][x], w_dq(d), r, TOKA ? x : h, sc2[j],
+                                                        nz2[j]);
+                        else
+                            dequant_w2(pk[j][x], w_dq(d), r, h);
+                    }
                     if constexpr (per_slab_handoff(BN)) {
                         // this slab's upcast stores become visible to the tensor core (async
                         // proxy), then one arrival per warp hands the buffer over
@@ -693,7 +722,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         const bool pairs = (N & 1) == 0;
         int j = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
             if (w.nk == 0) continue;
             const int b = j & 1;
             bool ok = mbar_wait(accf_bar(b), (j >> 1) & 1, abort_flag, err);
@@ -701,40 +730,85 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             // tcgen05.ld is warp-collective: decide per warp, never per lane
             ok = __all_sync(0xffffffffu, ok && !*abort_flag);
             if (!ok) break;
-            const int n = w.n0 + r;
-            // int8 requantisation (int32 modes): this lane's output-channel multiplier
-            const float rq = (T::c_bytes == 4 && mult && n < N) ? mult[n] : 0.f;
-            const uint32_t lane_addr =
-                tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
+            if constexpr (TOKA) {
+                // token-major: TMEM lane = token, columns = the tile's 256 weight rows, so each
+                // thread's results are contiguous in C (row t); tcgen05.ld stays warp-wide
+                const int t = w.t0 + tid;
+                const uint32_t lane_addr =
+                    tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * NMMA);
+                const bool vec16 = (N & 7) == 0;
+                if (w.t0 + warp * 32 < M) {
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 16) {
-                if (w.t0 + c >= M) break;
-                uint32_t v[16];
-                tmem_ld16(lane_addr + c, v);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int t = w.t0 + c + e;           // the same in every lane
-                    if (t >= M) break;
-                    if constexpr (T::c_bytes == 2) {
-                        // fp16 results leave as (n, n+1) pairs from neighbouring lanes
-                        const float x = __uint_as_float(v[e]);
-                        const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+                    for (int c = 0; c < NMMA; c += 16) {
+                        const int n = w.n0 + c;
+                        if (n >= N) break;
+                        uint32_t v[16];
+                        tmem_ld16(lane_addr + c, v);
+                        if (t >= M) continue;
                         __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
-                        if (pairs) {
-                            if ((lane & 1) == 0 && n < N) {
-                                const uint32_t h2 = pack_half2_rn(x, y);
-                                if (atomic_out) red_add_f16x2(dst, h2);
-                                else *reinterpret_cast<uint32_t *>(dst) = h2;
+                        uint32_t h2[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            h2[i] = pack_half2_rn(__uint_as_float(v[2 * i]),
+                                                  __uint_as_float(v[2 * i + 1]));
+                        if (n + 16 <= N && pairs) {
+                            if (atomic_out) {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) red_add_f16x2(dst + 2 * i, h2[i]);
+                            } else if (vec16) {
+                                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+                                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(h2[4], h2[5], h2[6], h2[7]);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) reinterpret_cast<uint32_t *>(dst)[i] = h2[i];
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                if (n + e >= N) break;
+                                const float x = __uint_as_float(v[e]);
+                                if (atomic_out) red_add_f16(dst + e, half_bits_rn(x));
+                                else dst[e] = __float2half_rn(x);
+                            }
+                        }
+                    }
+                }
+            } else {
+                const int n = w.n0 + r;
+                // int8 requantisation (int32 modes): this lane's output-channel multiplier
+                const float rq = (T::c_bytes == 4 && mult && n < N) ? mult[n] : 0.f;
+                const uint32_t lane_addr =
+                    tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 16) {
+                    if (w.t0 + c >= M) break;
+                    uint32_t v[16];
+                    tmem_ld16(lane_addr + c, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int t = w.t0 + c + e;           // the same in every lane
+                        if (t >= M) break;
+                        if constexpr (T::c_bytes == 2) {
+                            // fp16 results leave as (n, n+1) pairs from neighbouring lanes
+                            const float x = __uint_as_float(v[e]);
+                            const float y = __shfl_xor_sync(0xffffffffu, x, 1);
+                            __half *dst = static_cast<__half *>(C) + (size_t)t * N + n;
+                            if (pairs) {
+                                if ((lane & 1) == 0 && n < N) {
+                                    const uint32_t h2 = pack_half2_rn(x, y);
+                                    if (atomic_out) red_add_f16x2(dst, h2);
+                                    else *reinterpret_cast<uint32_t *>(dst) = h2;
+                                }
+                            } else if (n < N) {
+                                if (atomic_out) red_add_f16(dst, half_bits_rn(x));
+                                else *dst = __float2half_rn(x);
                             }
                         } else if (n < N) {
-                            if (atomic_out) red_add_f16(dst, half_bits_rn(x));
-                            else *dst = __float2half_rn(x);
+                            const size_t idx = (size_t)t * N + n;
+                            if (mult) static_cast<int8_t *>(C)[idx] = requant_i8((int)v[e], rq);
+                            else if (atomic_out) red_add_s32(static_cast<int32_t *>(C) + idx, (int)v[e]);
+                            else static_cast<int32_t *>(C)[idx] = (int)v[e];
                         }
-                    } else if (n < N) {
-                        const size_t idx = (size_t)t * N + n;
-                        if (mult) static_cast<int8_t *>(C)[idx] = requant_i8((int)v[e], rq);
-                        else if (atomic_out) red_add_s32(static_cast<int32_t *>(C) + idx, (int)v[e]);
-                        else static_cast<int32_t *>(C)[idx] = (int)v[e];
                     }
                 }
             }
@@ -768,31 +842,31 @@ int mode_of(int op)
     }
 }
 
-int smem_bytes(int mode, int bn, int stages, int pg)
+int smem_bytes(int mode, int bn, int stages, int pg, int wr = kRowsW)
 {
     const bool packed = (is_w4(mode) || mode == kW2A8);
-    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg), pg,
-                      packed ? packed_stages(pg, bn, stages) : 0);
+    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg, wr), pg,
+                      packed ? packed_stages(pg, bn, stages, wr) : 0, wr);
 }
 
 // slabs per packed-weight copy for this problem and tile: 4 when K holds a whole number of
 // 4-slab runs and that plan fits in shared memory, else 1
-int packed_group(const Problem &p, int bn, int stages)
+int packed_group(const Problem &p, int bn, int stages, int wr = kRowsW)
 {
     const int mode = mode_of(p.op);
     if (!(is_w4(mode) || mode == kW2A8)) return 1;
     const int kps = is_w4(mode) ? 64 : 128;
     if (p.K % kps || (p.K / kps) % 4) return 1;
-    return smem_bytes(mode, bn, stages, 4) <= kMaxSmem ? 4 : 1;
+    return smem_bytes(mode, bn, stages, 4, wr) <= kMaxSmem ? 4 : 1;
 }
 
-template <int MODE, int BN, int STAGES, int PG>
+template <int MODE, int BN, int STAGES, int PG, bool TOKA = false>
 cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES, PG>;
+    using L = Smem<MODE, BN, STAGES, PG, TOKA>;
     if (L::total > kMaxSmem) return cudaErrorInvalidConfiguration;
-    auto kern = tc_gemm_kernel<MODE, BN, STAGES, PG>;
+    auto kern = tc_gemm_kernel<MODE, BN, STAGES, PG, TOKA>;
     // the dynamic shared-memory opt-in is per device: remember it per device
     static std::mutex mu;
     static bool opted_in[64] = {};
@@ -822,7 +896,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                       CU_TENSOR_MAP_SWIZZLE_128B);
     } else if constexpr (is_w4(MODE)) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
-                      8 * PG, kRowsW, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
+                      8 * PG, L::WR, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
                       BN, CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
@@ -836,7 +910,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     const int nkb = (p.K + T::k_per_slab - 1) / T::k_per_slab;
     const int kbps = ((nkb + split_k - 1) / split_k + PG - 1) / PG * PG;   // whole copies
     const int splits = (nkb + kbps - 1) / kbps;
-    const int n_tiles = (p.N + kRowsW - 1) / kRowsW;
+    const int n_tiles = (p.N + L::WR - 1) / L::WR;
     const int t_tiles = (p.M + BN - 1) / BN;
     const long units = (long)n_tiles * t_tiles * splits;
     if (units > 0x7fffffffL) return cudaErrorInvalidValue;
@@ -850,7 +924,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                 cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return cudaErrorInvalidConfiguration;
-        occ = std::min(occ, (int)(512 / tmem_cols<BN>()));
+        occ = std::min(occ, (int)(512 / tmem_cols<TOKA ? kRowsT : BN>()));
         sm_count[dev] = sms;
         per_sm[dev] = std::max(1, occ);
     }
@@ -891,6 +965,23 @@ cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned in
     return launch_stages_pg<MODE, BN, 1>(p, c, err, stream);
 }
 
+// token-major variant (swap_ab = 0): tiles of 128 tokens x 256 weight rows, W4A16 only
+template <int MODE>
+cudaError_t launch_toka(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                        cudaStream_t stream)
+{
+    const bool g4 = packed_group(p, kTokT, c.stages, kRowsT) == 4;
+    switch (c.stages) {
+    case 2: return g4 ? launch_t<MODE, kTokT, 2, 4, true>(p, c.split_k, err, stream)
+                      : launch_t<MODE, kTokT, 2, 1, true>(p, c.split_k, err, stream);
+    case 3: return g4 ? launch_t<MODE, kTokT, 3, 4, true>(p, c.split_k, err, stream)
+                      : launch_t<MODE, kTokT, 3, 1, true>(p, c.split_k, err, stream);
+    case 4: return g4 ? launch_t<MODE, kTokT, 4, 4, true>(p, c.split_k, err, stream)
+                      : launch_t<MODE, kTokT, 4, 1, true>(p, c.split_k, err, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int MODE>
 cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                       cudaStream_t stream)
@@ -910,6 +1001,15 @@ cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *e
 bool tc_supports(const Problem &p, const qgemm_config_t &c)
 {
     if (c.path != QG_PATH_TC) return false;
+    if (!c.swap_ab) {
+        // token-major variant: W4A16 with scale groups of whole slabs
+        if (p.op != QG_OP_W4A16 || c.bm != kTokT || c.bn != kRowsT) return false;
+        if (c.stages < 2 || c.stages > 4 || c.split_k < 1 || c.split_k > 64) return false;
+        if (p.K % 64 || p.gs % 64 || p.K % p.gs) return false;
+        const int pg = packed_group(p, kTokT, c.stages, kRowsT);
+        return smem_bytes(kW4A16, kTokT, c.stages, pg, kRowsT) <= kMaxSmem &&
+               dq_buffers(true, kTokT, c.stages, pg, kRowsT) >= 3;
+    }
     if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
     if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 128 && c.stages == 8) ||
           (c.bn <= 64 && c.stages == 16)))
@@ -950,6 +1050,11 @@ int tc_max_stages(const Problem &p, int bn)
 cudaError_t launch_tc(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                       cudaStream_t stream)
 {
+    if (!c.swap_ab) {
+        if (p.op != QG_OP_W4A16) return cudaErrorInvalidValue;
+        return p.interleaved ? launch_toka<kW4A16I>(p, c, err, stream)
+                             : launch_toka<kW4A16>(p, c, err, stream);
+    }
     switch (mode_of(p.op)) {
     case kDense: return launch_bn<kDense>(p, c, err, stream);
     case kW8A8: return launch_bn<kW8A8>(p, c, err, stream);

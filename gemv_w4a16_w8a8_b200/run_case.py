@@ -36,6 +36,8 @@ def main(argv=None) -> int:
     ap.add_argument("--stages", type=int, default=-1)
     ap.add_argument("--bk", type=int, default=0)
     ap.add_argument("--bm", type=int, default=0, help="TC: tile M; STREAM: warps per CTA")
+    ap.add_argument("--swap-ab", type=int, default=-1,
+                    help="TC: 1 = weights in the MMA's M side, 0 = token-major tile")
     ap.add_argument("--copies", type=int, default=0, help="weight copies (0: >= 3x L2)")
     a = ap.parse_args(argv)
 
@@ -77,7 +79,7 @@ def main(argv=None) -> int:
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + 2 * M * K + 2 * M * N
 
-    if a.path or a.rows or a.bn or a.bk or a.bm or a.stages >= 0:
+    if a.path or a.rows or a.bn or a.bk or a.bm or a.stages >= 0 or a.swap_ab >= 0:
         cfg = qg.qgemm_plan(opc, M, N, K, gs, hz)
         if a.path and a.path != cfg["path"]:
             cfg = {k: 0 for k in cfg}
@@ -88,6 +90,8 @@ def main(argv=None) -> int:
                 cfg[key] = val
         if a.stages >= 0:
             cfg["stages"] = a.stages
+        if a.swap_ab >= 0:
+            cfg["swap_ab"] = a.swap_ab
         qg.qgemm_set_config(opc, M, N, K, gs, hz, cfg)
     print("config", qg.qgemm_plan(opc, M, N, K, gs, hz, a.split_k))
 

@@ -87,12 +87,16 @@ typedef enum qg_path {
 typedef struct qgemm_config_t {
     int32_t path;    /* qg_path                                                             */
     int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise)  */
-    int32_t bm;      /* TC: tile extent along M                                              */
-    int32_t bn;      /* TC: tile extent along N                                              */
+    int32_t bm;      /* TC: tile extent along the MMA's M (128)                              */
+    int32_t bn;      /* TC: tile extent along the MMA's N                                    */
     int32_t bk;      /* TC: tile extent along K                                              */
-    int32_t stages;  /* TC: activation ring depth (2..5; also 8, 16 for bn <= 64)           */
+    int32_t stages;  /* TC: activation ring depth (2..5; 8 for bn <= 128, 16 for bn <= 64;
+                        2..4 when swap_ab = 0)                                               */
     int32_t split_k; /* number of K parts (1 = no atomics)                                   */
-    int32_t swap_ab; /* TC: 1 = weights fill the MMA's M side, tokens its N side             */
+    int32_t swap_ab; /* TC: 1 = weights fill the MMA's M side (bm = 128 weight rows), tokens
+                        its N side (bn = 16..256 tokens); 0 = token-major, W4A16 with a group
+                        size that is a multiple of 64: bm = 128 tokens, bn = 256 weight rows
+                        (an MMA from shared memory reaches its full rate only at N = 256)    */
 } qgemm_config_t;
 
 /* ---- matmuls ----------------------------------------------------------------------------- */

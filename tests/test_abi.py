@@ -195,8 +195,16 @@ def test_plan_large_m_uses_tensor_cores():
     c = qg.qgemm_plan(qg.OP_W4A16, 16384, 16384, 16384, 128, 1)
     assert c["path"] == qg.PATH_TC and c["bn"] == 256 and 2 <= c["stages"] <= 5
     assert c["split_k"] == 1                     # 8192 tiles fill the GPU many times
+    c = qg.qgemm_plan(qg.OP_W4A16, 16384, 16384, 16384, 128, 1)
+    assert c["swap_ab"] == 1                     # weights in the MMA's M side
+    # up to one tile of tokens: the token-major tile (128 tokens x 256 weight rows), K split
+    # until the units fill the GPU
     c = qg.qgemm_plan(qg.OP_W4A16, 32, 16384, 16384, 128, 1)
-    assert c["path"] == qg.PATH_TC and c["bn"] == 32 and c["split_k"] >= 1
+    assert c["path"] == qg.PATH_TC and c["swap_ab"] == 0 and (c["bm"], c["bn"]) == (128, 256)
+    assert c["split_k"] >= 2 and 2 <= c["stages"] <= 4
+    # group size 32 (not whole slabs) keeps the weight-major tile
+    c = qg.qgemm_plan(qg.OP_W4A16, 32, 16384, 16384, 32, 1)
+    assert c["path"] == qg.PATH_TC and c["swap_ab"] == 1 and c["bn"] == 32
     c = qg.qgemm_plan(qg.OP_DENSE_F16, 1, 256, 256)
     assert c["path"] == qg.PATH_TC and c["bn"] == 16
     for op in (qg.OP_W8A8, qg.OP_W2A8):

@@ -36,6 +36,20 @@ def tc_config(op, M, N, K, gs, hz, bn, stages, split_k):
         qg.qgemm_set_config(OPS[op], M, N, K, gs, hz, None)
 
 
+@contextlib.contextmanager
+def toka_config(M, N, K, gs, hz, stages, split_k):
+    """Pin the token-major tensor-core tile (128 tokens x 256 weight rows, W4A16)."""
+    cfg = {"path": qg.PATH_TC, "rows": 0, "bm": 128, "bn": 256, "bk": 0, "stages": stages,
+           "split_k": split_k, "swap_ab": 0}
+    qg.qgemm_set_config(qg.OP_W4A16, M, N, K, gs, hz, cfg)
+    try:
+        plan = qg.qgemm_plan(qg.OP_W4A16, M, N, K, gs, hz)
+        assert plan["path"] == qg.PATH_TC and plan["swap_ab"] == 0
+        yield
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, M, N, K, gs, hz, None)
+
+
 class DenseCase:
     def __init__(self, M, N, K, seed=0):
         self.M, self.N, self.K = M, N, K
@@ -141,6 +155,67 @@ def test_w4a16_tc_long_k_deep_rings(bn, stages, split_k):
         assert_fp16_close(case.run(), case.ref_full(), f"bn={bn} st={stages} split={split_k}")
 
 
+# ---- W4A16, token-major tiles (tokens in the MMA's M, 256 weight rows in its N) ----------------
+
+TOKA_SHAPES = [(1, 256, 256, 64, 1), (8, 384, 1024, 128, 0), (17, 136, 512, 128, 1),
+               (100, 1000, 2048, 128, 1), (128, 256, 1024, -1, 1), (129, 520, 768, 64, 0),
+               (200, 257, 1024, 128, 1), (64, 4104, 1152, 128, 1)]
+
+
+@pytest.mark.parametrize("M,N,K,gs,hz", TOKA_SHAPES)
+@pytest.mark.parametrize("stages,split_k", [(2, 1), (3, 1), (4, 1), (4, 3), (2, 16)])
+def test_w4a16_toka_tiles(M, N, K, gs, hz, stages, split_k):
+    """Ragged tokens (rows past M read as zero), ragged weight tiles (N % 256, N odd, N % 8),
+    single-slab packed copies (K = 768, 1152) and K splits."""
+    case = W4Case(M, N, K, gs, hz, seed=M * 5 + N + K)
+    try:
+        cm = toka_config(M, N, K, gs, hz, stages, split_k)
+        cm.__enter__()
+    except qg.QGemmError:
+        pytest.skip(f"stages={stages} does not fit K={K}")
+    try:
+        assert_fp16_close(case.run(), case.ref_full(), f"toka {M},{N},{K} gs={gs} st={stages}")
+    finally:
+        cm.__exit__(None, None, None)
+
+
+def test_w4a16_toka_guard_bands_and_stream():
+    M, N, K = 77, 520, 1024
+    case = W4Case(M, N, K, 128, 1, seed=21)
+    buf, C, pad = guarded((M, N), torch.float16)
+    s = torch.cuda.Stream()
+    with toka_config(M, N, K, 128, 1, 4, 3), torch.cuda.stream(s):
+        case.run(C=C)
+    s.synchronize()
+    assert guards_intact(buf, pad, M * N)
+    assert_fp16_close(C, case.ref_full(), "toka guarded")
+
+
+def test_w4a16_toka_one_hot_element_order():
+    """A = e_k (token k reads weight column k): C[k, n] = fp16((q - z) s) for every k and n."""
+    N, K, gs = 300, 128, 64
+    G = K // gs
+    codes = synth.uniform_int((N, K), 0, 15, 13, synth.TID_W, np.uint8)
+    s = synth.uniform_f16((N, G), 0.001, 0.01, 13, synth.TID_SCALE)
+    z = synth.uniform_int((N, G), 0, 15, 13, synth.TID_ZERO, np.uint8).astype(np.float16)
+    A = np.eye(K, dtype=np.float16)
+    with toka_config(K, N, K, gs, 1, 2, 1):
+        C = qg.qgemm_w4a16(to_dev(A), qg.quant_pack_int4(to_dev(codes)), to_dev(s), to_dev(z),
+                           group_size=gs).cpu().numpy()
+    ref = oracle.w4a16(A, oracle.pack_int4(codes), s, z, K, gs)
+    assert_fp16_close(torch.from_numpy(C.astype(np.float32)), ref, "toka one-hot")
+
+
+@pytest.mark.parametrize("M", [1, 16, 32, 128])
+def test_w4a16_toka_full_size_sampled(M):
+    N = K = 16384
+    case = W4Case(M, N, K, 128, 1, seed=M + 70)
+    with toka_config(M, N, K, 128, 1, 4, 16):
+        C = case.run().float().cpu().numpy()
+    ms, ns = sample_pairs(M, N, 300, seed=M + 1)
+    assert_fp16_close(torch.from_numpy(C[ms, ns]), case.ref_at(ms, ns), f"toka M={M}")
+
+
 @pytest.fixture(scope="module")
 def copy_tagged_weights():
     """N = K = 16384 weights whose codes name their position: every weight of 256-wide K
@@ -158,8 +233,10 @@ def copy_tagged_weights():
     return Wq, S, Z, row
 
 
+# bn = 0: the token-major tile
 @pytest.mark.parametrize("bn,stages,split_k", [(16, 16, 1), (32, 16, 1), (32, 16, 2), (32, 4, 2),
-                                               (64, 8, 1), (128, 8, 2), (256, 4, 1)])
+                                               (64, 8, 1), (128, 8, 2), (256, 4, 1), (0, 2, 1),
+                                               (0, 4, 1), (0, 4, 16), (0, 3, 5)])
 def test_w4a16_tc_packed_ring_positions(copy_tagged_weights, bn, stages, split_k):
     """Token m reads exactly one slab (slab 4m + m % 4: every packed copy once, at every position
     inside it), so each output is 64 x the code of the copy the MMA actually used; compared
@@ -172,7 +249,9 @@ def test_w4a16_tc_packed_ring_positions(copy_tagged_weights, bn, stages, split_k
     ref = oracle.w4a16(A, row, ones, zeros, K, 128)                  # one weight row: [M, 1]
     assert np.array_equal(ref[:, 0], 64.0 * ((slab // 4) % 16))
     Ad = to_dev(A)
-    with tc_config("w4a16", M, N, K, 128, 1, bn, stages, split_k):
+    cfg = toka_config(M, N, K, 128, 1, stages, split_k) if bn == 0 else \
+        tc_config("w4a16", M, N, K, 128, 1, bn, stages, split_k)
+    with cfg:
         for _ in range(3):
             C = qg.qgemm_w4a16(Ad, Wq, S, Z, group_size=128).cpu().numpy().astype(np.float64)
             bad = np.argwhere(C != ref)
