@@ -194,6 +194,7 @@ qgemm_config_t tc_default(const Problem &p, int sms)
     c.bm = 128;
     c.bn = pow2_at_least(p.M, 16, 256);
     c.bk = k_per_slab(p.op);
+    c.swap_ab = 1;
     // packed weights: the deepest ring that still leaves three dequant buffers (four for token
     // tiles of 128 and more, which hand them over slab by slab; both measured faster than a
     // deeper activation ring with fewer); other ops: the deepest ring that fits
@@ -471,6 +472,19 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                     c.split_k = s;
                     if (supports(p, c)) out.push_back(c);
                 }
+        if (p.op == QG_OP_W4A16 && p.M == 1) {
+            // one token on the FMA pipe (TMA-fed kernel, bn = 1)
+            for (int rows : {32, 64, 128})
+                for (int st : {2, 3, 4, 6})
+                    for (int s = 1; s <= 16; s *= 2) {
+                        c.rows = rows;
+                        c.bn = 1;
+                        c.stages = st;
+                        c.split_k = s;
+                        if (supports(p, c)) out.push_back(c);
+                    }
+            c.bn = 0;
+        }
     }
     if (p.op == QG_OP_W4A16 && p.M <= 16) {
         // every stage shape and warp split, each at its deepest ring and at two-thirds of it

@@ -314,7 +314,7 @@ void launch_nt(const Problem &p, int rows, int split_k, cudaStream_t stream)
 
 bool gemv_w4a16_supports(const Problem &p, const qgemm_config_t &cfg)
 {
-    return p.K % 32 == 0 && p.gs % 32 == 0 && p.K % p.gs == 0 && cfg.stages == 0 &&
+    return p.K % 32 == 0 && p.gs % 32 == 0 && p.K % p.gs == 0 && cfg.stages == 0 && cfg.bn == 0 &&
            (cfg.rows == 16 || cfg.rows == 32 || cfg.rows == 64) && cfg.split_k >= 1 &&
            cfg.split_k <= 64;
 }

@@ -15,6 +15,12 @@
 //     corr = sum_k c_k a_k and, in rows 8..15, sum_k a_k. Then per k-block, in fp32,
 //         sum_k a_k (q_k - z) s = s * (D - corr - z * sum_k a_k).
 //     Five instructions upcast eight codes; the MMA pipe absorbs the rest.
+// SIMT variant for one token: the warp-level MMA issues at ~9 cycles per m16n8k16 on sm_100,
+// which caps a one-token GEMV near 3 TB/s. With one token each lane instead multiplies the same
+// biased codes x with its activation pairs by mixed-precision FMAs (fp16 inputs, fp32
+// accumulate: every product exact), so the same five instructions plus eight FMAs handle eight
+// codes; the bias sum_k c_k a_k and sum_k a_k of the lane's 32-wide K quarter are shared by all
+// its rows and split over the eight lanes that hold the same quarter.
 #include <mutex>
 
 #include "sm100.cuh"
@@ -45,6 +51,17 @@ __device__ __forceinline__ void act_pairs_scaled(const uint4 &v, uint32_t (&b)[4
     }
 }
 
+// acc + x.lo * a.lo + x.hi * a.hi, both products exact in fp32 (fp16 x fp16), two roundings
+__device__ __forceinline__ float fma2_f16_f32(uint32_t x, uint32_t a, float acc)
+{
+    asm("{\n\t.reg .f16 xl, xh, al, ah;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\tmov.b32 {al, ah}, %2;\n\t"
+        "fma.rn.f32.f16 %0, xl, al, %0;\n\tfma.rn.f32.f16 %0, xh, ah, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(x), "r"(a));
+    return acc;
+}
+
 template <int RB, int NT, int STAGES> struct Layout {
     static constexpr int rows = 16 * RB;
     static constexpr int slot = rows * 64;             // one stage: rows x 16 packed words
@@ -56,7 +73,8 @@ template <int RB, int NT, int STAGES> struct Layout {
 };
 
 // RB: 16-row blocks per CTA (all four warps share them and split K).  NT: 8-token tiles.
-template <int RB, int NT, int STAGES, bool ILV>
+// SIMT: one token, products on the FMA pipe instead of the warp-level MMA (NT = 1, M = 1).
+template <int RB, int NT, int STAGES, bool ILV, bool SIMT = false>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__restrict__ A,
                       const __half *__restrict__ S, const __half *__restrict__ Z,
@@ -113,7 +131,8 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
     bool aok[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
-        const int tok = tok0 + 8 * t + lg;
+        // MMA fragments: lane group lg holds token lg; SIMT: every lane holds the one token
+        const int tok = SIMT ? tok0 : tok0 + 8 * t + lg;
         aok[t] = tok < M;
         arow[t] = A + (size_t)min(tok, M - 1) * K + 32 * lt;
     }
@@ -173,60 +192,110 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
             }
         if (i + 1 < cnt) prefetch(i + 1);
         if (!mbar_wait(smem_u32(&full[warp][s]), (i / STAGES) & 1, abort_v, err)) break;
-        // two independent accumulation chains per product keep the MMA pipe busy
-        float cz[NT][4], cz2[NT][4];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) cz[t][e] = cz2[t][e] = 0.f;
+        if constexpr (SIMT) {
+            static_assert(NT == 1, "the SIMT inner product serves one token");
+            // sum_k c_k a_k / 1024 and sum_k a_k of this lane's K quarter: the eight lanes that
+            // hold the quarter (lane = 4 rq + lt) take two of its sixteen pairs each
+            const int rq = lg;
+            // (a, a') at weight 1 and (a / 16, a' / 16); picked with masks, not an index, so
+            // that b stays in registers
+            uint32_t pe = 0u, po = 0u;
+            const uint32_t odd = 0u - (uint32_t)(rq & 1);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                mma_16816_f16(cz[t], kones, b[t][j][0], b[t][j][1], cz[t]);
-                mma_16816_f16(cz2[t], kones, b[t][j][2], b[t][j][3], cz2[t]);
+                const uint32_t mj = 0u - (uint32_t)((rq >> 1) == j);
+                pe |= mj & ((b[0][j][2] & odd) | (b[0][j][0] & ~odd));
+                po |= mj & ((b[0][j][3] & odd) | (b[0][j][1] & ~odd));
             }
+            const float2 fe = __half22float2(*reinterpret_cast<const __half2 *>(&pe));
+            const float2 fo = __half22float2(*reinterpret_cast<const __half2 *>(&po));
+            float csum = (fe.x + fe.y) + (fo.x + fo.y);
+            float asum = (fe.x + fe.y) + 16.f * (fo.x + fo.y);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cz[t][e] += cz2[t][e];
-        }
-        const uint8_t *slot = &ring[warp][s][0];
+            for (int m = 4; m < 32; m <<= 1) {
+                csum += __shfl_xor_sync(0xffffffffu, csum, m);
+                asum += __shfl_xor_sync(0xffffffffu, asum, m);
+            }
+            const float corr = 1024.f * csum;
+            const uint8_t *slot = &ring[warp][s][0];
 #pragma unroll
-        for (int r = 0; r < RB; ++r) {
-            const uint4 wa = *reinterpret_cast<const uint4 *>(slot + (16 * r + lg) * 64 + 16 * lt);
-            const uint4 wb =
-                *reinterpret_cast<const uint4 *>(slot + (16 * r + lg + 8) * 64 + 16 * lt);
-            const uint32_t wva[4] = {wa.x, wa.y, wa.z, wa.w};
-            const uint32_t wvb[4] = {wb.x, wb.y, wb.z, wb.w};
-            float d[NT][4], d2[NT][4];
+            for (int r = 0; r < RB; ++r) {
+                const uint4 wa = *reinterpret_cast<const uint4 *>(slot + (16 * r + lg) * 64 + 16 * lt);
+                const uint4 wb =
+                    *reinterpret_cast<const uint4 *>(slot + (16 * r + lg + 8) * 64 + 16 * lt);
+                const uint32_t wv[2][4] = {{wa.x, wa.y, wa.z, wa.w}, {wb.x, wb.y, wb.z, wb.w}};
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
+                for (int h = 0; h < 2; ++h) {
+                    float p0 = 0.f, p1 = 0.f;   // two chains
 #pragma unroll
-                for (int e = 0; e < 4; ++e) d[t][e] = d2[t][e] = 0.f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
-                const uint32_t xa = wva[j], xb = wvb[j];
-                const uint32_t xa8 = xa >> 8, xb8 = xb >> 8;
-                const uint32_t a0[4] = {lop3_and_or(xa, kLo, kMagic), lop3_and_or(xb, kLo, kMagic),
-                                        lop3_and_or(xa, kHi, kMagic), lop3_and_or(xb, kHi, kMagic)};
-                const uint32_t a1[4] = {lop3_and_or(xa8, kLo, kMagic), lop3_and_or(xb8, kLo, kMagic),
-                                        lop3_and_or(xa8, kHi, kMagic), lop3_and_or(xb8, kHi, kMagic)};
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    mma_16816_f16(d[t], a0, b[t][j][0], b[t][j][1], d[t]);
-                    mma_16816_f16(d2[t], a1, b[t][j][2], b[t][j][3], d2[t]);
+                    for (int j = 0; j < 4; ++j) {
+                        constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
+                        const uint32_t x = wv[h][j], x8 = x >> 8;
+                        p0 = fma2_f16_f32(lop3_and_or(x, kLo, kMagic), b[0][j][0], p0);
+                        p1 = fma2_f16_f32(lop3_and_or(x, kHi, kMagic), b[0][j][1], p1);
+                        p0 = fma2_f16_f32(lop3_and_or(x8, kLo, kMagic), b[0][j][2], p0);
+                        p1 = fma2_f16_f32(lop3_and_or(x8, kHi, kMagic), b[0][j][3], p1);
+                    }
+                    // rows 16 r + lg (+ 8): this lane's part of s * (sum a q - z sum a)
+                    acc[r][0][2 * h] += sc[r][h] * ((p0 + p1) - corr - zr[r][h] * asum);
                 }
             }
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) d[t][e] += d2[t][e];
-            // d0 (row g, tok 2t) d1 (row g, tok 2t+1) d2 (row g+8, tok 2t) d3 (row g+8, 2t+1)
-            // cz0/cz1: corr of tok 2t / 2t+1;  cz2/cz3: sum a of tok 2t / 2t+1
+        } else {
+            // two independent accumulation chains per product keep the MMA pipe busy
+            float cz[NT][4], cz2[NT][4];
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                acc[r][t][0] += sc[r][0] * (d[t][0] - cz[t][0] - zr[r][0] * cz[t][2]);
-                acc[r][t][1] += sc[r][0] * (d[t][1] - cz[t][1] - zr[r][0] * cz[t][3]);
-                acc[r][t][2] += sc[r][1] * (d[t][2] - cz[t][0] - zr[r][1] * cz[t][2]);
-                acc[r][t][3] += sc[r][1] * (d[t][3] - cz[t][1] - zr[r][1] * cz[t][3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cz[t][e] = cz2[t][e] = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_16816_f16(cz[t], kones, b[t][j][0], b[t][j][1], cz[t]);
+                    mma_16816_f16(cz2[t], kones, b[t][j][2], b[t][j][3], cz2[t]);
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cz[t][e] += cz2[t][e];
+            }
+            const uint8_t *slot = &ring[warp][s][0];
+#pragma unroll
+            for (int r = 0; r < RB; ++r) {
+                const uint4 wa = *reinterpret_cast<const uint4 *>(slot + (16 * r + lg) * 64 + 16 * lt);
+                const uint4 wb =
+                    *reinterpret_cast<const uint4 *>(slot + (16 * r + lg + 8) * 64 + 16 * lt);
+                const uint32_t wva[4] = {wa.x, wa.y, wa.z, wa.w};
+                const uint32_t wvb[4] = {wb.x, wb.y, wb.z, wb.w};
+                float d[NT][4], d2[NT][4];
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d[t][e] = d2[t][e] = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
+                    const uint32_t xa = wva[j], xb = wvb[j];
+                    const uint32_t xa8 = xa >> 8, xb8 = xb >> 8;
+                    const uint32_t a0[4] = {lop3_and_or(xa, kLo, kMagic), lop3_and_or(xb, kLo, kMagic),
+                                            lop3_and_or(xa, kHi, kMagic), lop3_and_or(xb, kHi, kMagic)};
+                    const uint32_t a1[4] = {lop3_and_or(xa8, kLo, kMagic), lop3_and_or(xb8, kLo, kMagic),
+                                            lop3_and_or(xa8, kHi, kMagic), lop3_and_or(xb8, kHi, kMagic)};
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        mma_16816_f16(d[t], a0, b[t][j][0], b[t][j][1], d[t]);
+                        mma_16816_f16(d2[t], a1, b[t][j][2], b[t][j][3], d2[t]);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) d[t][e] += d2[t][e];
+                // d0 (row g, tok 2t) d1 (row g, tok 2t+1) d2 (row g+8, tok 2t) d3 (row g+8, 2t+1)
+                // cz0/cz1: corr of tok 2t / 2t+1;  cz2/cz3: sum a of tok 2t / 2t+1
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    acc[r][t][0] += sc[r][0] * (d[t][0] - cz[t][0] - zr[r][0] * cz[t][2]);
+                    acc[r][t][1] += sc[r][0] * (d[t][1] - cz[t][1] - zr[r][0] * cz[t][3]);
+                    acc[r][t][2] += sc[r][1] * (d[t][2] - cz[t][0] - zr[r][1] * cz[t][2]);
+                    acc[r][t][3] += sc[r][1] * (d[t][3] - cz[t][1] - zr[r][1] * cz[t][3]);
+                }
             }
         }
         consumed = i + 1;
@@ -245,6 +314,18 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
     }
 
     // ---- block reduction of the four warps, then store / atomic add -------------------------
+    if constexpr (SIMT) {
+        // acc[r][0][0] / [2]: rows 16 r + lg / 16 r + lg + 8, this lane's K quarter lt
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                float v = acc[r][0][e];
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                if (lt == 0) red[warp][0][16 * r + lg + 4 * e] = v;
+            }
+    } else
 #pragma unroll
     for (int r = 0; r < RB; ++r)
 #pragma unroll
@@ -318,12 +399,12 @@ gemv_w4a16_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const __half *__
     }
 }
 
-template <int RB, int NT, int STAGES, bool ILV>
+template <int RB, int NT, int STAGES, bool ILV, bool SIMT = false>
 cudaError_t launch_ilv(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
                        float *ws_part, unsigned int *ws_count)
 {
     using L = Layout<RB, NT, STAGES>;
-    auto kern = gemv_w4a16_tma_kernel<RB, NT, STAGES, ILV>;
+    auto kern = gemv_w4a16_tma_kernel<RB, NT, STAGES, ILV, SIMT>;
     static std::mutex mu;
     static bool opted_in[64] = {};
     int dev = 0;
@@ -352,13 +433,26 @@ cudaError_t launch_ilv(const Problem &p, int split_k, unsigned int *err, cudaStr
     return cudaGetLastError();
 }
 
-template <int RB, int NT, int STAGES>
+template <int RB, int NT, int STAGES, bool SIMT = false>
 cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
                        float *ws_part, unsigned int *ws_count)
 {
-    return p.interleaved ? launch_ilv<RB, NT, STAGES, true>(p, split_k, err, stream, ws_part, ws_count)
-                         : launch_ilv<RB, NT, STAGES, false>(p, split_k, err, stream, ws_part,
-                                                             ws_count);
+    return p.interleaved
+               ? launch_ilv<RB, NT, STAGES, true, SIMT>(p, split_k, err, stream, ws_part, ws_count)
+               : launch_ilv<RB, NT, STAGES, false, SIMT>(p, split_k, err, stream, ws_part, ws_count);
+}
+
+// one token on the FMA pipe (config bn = 1): 32, 64 or 128 rows per CTA
+template <int RB>
+cudaError_t launch_simt_stages(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                               cudaStream_t stream, float *wp, unsigned int *wc)
+{
+    switch (c.stages) {
+    case 2: return launch_one<RB, 1, 2, true>(p, c.split_k, err, stream, wp, wc);
+    case 3: return launch_one<RB, 1, 3, true>(p, c.split_k, err, stream, wp, wc);
+    case 4: return launch_one<RB, 1, 4, true>(p, c.split_k, err, stream, wp, wc);
+    default: return launch_one<RB, 1, 6, true>(p, c.split_k, err, stream, wp, wc);
+    }
 }
 
 template <int RB, int NT>
@@ -386,14 +480,22 @@ cudaError_t launch_rb(const Problem &p, const qgemm_config_t &c, unsigned int *e
 
 bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &c)
 {
-    return p.gs % kKB == 0 && p.K % kKB == 0 && (c.rows == 16 || c.rows == 32 || c.rows == 64) &&
-           (c.stages == 2 || c.stages == 3 || c.stages == 4 || c.stages == 6) && c.split_k >= 1 &&
-           c.split_k <= 64;
+    const bool stages_ok = c.stages == 2 || c.stages == 3 || c.stages == 4 || c.stages == 6;
+    const bool base = p.gs % kKB == 0 && p.K % kKB == 0 && stages_ok && c.split_k >= 1 &&
+                      c.split_k <= 64;
+    if (c.bn == 1)   // one token on the FMA pipe
+        return base && p.M == 1 && (c.rows == 32 || c.rows == 64 || c.rows == 128);
+    return base && c.bn == 0 && (c.rows == 16 || c.rows == 32 || c.rows == 64);
 }
 
 cudaError_t launch_gemv_w4a16_tma(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                                   cudaStream_t stream, float *ws_part, unsigned int *ws_count)
 {
+    if (c.bn == 1) {
+        if (c.rows == 32) return launch_simt_stages<2>(p, c, err, stream, ws_part, ws_count);
+        if (c.rows == 64) return launch_simt_stages<4>(p, c, err, stream, ws_part, ws_count);
+        return launch_simt_stages<8>(p, c, err, stream, ws_part, ws_count);
+    }
     if (p.M <= 8) return launch_rb<1>(p, c, err, stream, ws_part, ws_count);
     return launch_rb<2>(p, c, err, stream, ws_part, ws_count);
 }

@@ -88,7 +88,8 @@ typedef struct qgemm_config_t {
     int32_t path;    /* qg_path                                                             */
     int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise)  */
     int32_t bm;      /* TC: tile extent along the MMA's M (128)                              */
-    int32_t bn;      /* TC: tile extent along the MMA's N                                    */
+    int32_t bn;      /* TC: tile extent along the MMA's N. GEMV (W4A16, stages > 0, M = 1):
+                        1 = products on the FMA pipe instead of the warp-level MMA           */
     int32_t bk;      /* TC: tile extent along K                                              */
     int32_t stages;  /* TC: activation ring depth (2..5; 8 for bn <= 128, 16 for bn <= 64;
                         2..4 when swap_ab = 0)                                               */

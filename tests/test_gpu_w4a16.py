@@ -75,6 +75,68 @@ def test_w4a16_each_row_tile(rows, M, stages):
         qg.qgemm_set_config(qg.OP_W4A16, M, 200, 1024, 128, 1, None)
 
 
+# ---- one token on the FMA pipe (TMA-fed GEMV, bn = 1) -------------------------------------------
+
+def simt_cfg(rows, stages, split_k):
+    return {"path": qg.PATH_GEMV, "rows": rows, "bm": 0, "bn": 1, "bk": 0, "stages": stages,
+            "split_k": split_k, "swap_ab": 0}
+
+
+SIMT_SHAPES = [(64, 128, 128, 1), (200, 1024, 128, 0), (4104, 4096, 256, 1), (513, 2048, -1, 1),
+               (4095, 1152, 128, 1), (130, 384, 384, 0)]
+
+
+@pytest.mark.parametrize("N,K,gs,hz", SIMT_SHAPES)
+@pytest.mark.parametrize("rows,stages,split_k", [(32, 2, 1), (64, 4, 3), (128, 6, 16),
+                                                 (128, 3, 1), (64, 2, 64)])
+def test_w4a16_simt_one_token(N, K, gs, hz, rows, stages, split_k):
+    """Ragged weight rows (N % rows), one-group K (gs = -1), group sizes 128 .. 384, K splits that
+    leave empty parts, each with and without zero points."""
+    case = W4Case(1, N, K, gs, hz, seed=N + K + rows)
+    ge = K if gs == -1 else gs
+    qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, ge, hz, simt_cfg(rows, stages, split_k))
+    try:
+        assert qg.qgemm_plan(qg.OP_W4A16, 1, N, K, ge, hz)["bn"] == 1
+        assert_fp16_close(case.run(), case.ref_full(), f"simt N={N} K={K} rows={rows}")
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, ge, hz, None)
+
+
+def test_w4a16_simt_rejects_more_tokens():
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_W4A16, 2, 256, 1024, 128, 1, simt_cfg(64, 4, 1))
+
+
+def test_w4a16_simt_one_hot_rows_and_fractional_zero():
+    """A = e_k for one k at a time (one token): C[0, n] = (q[n,k] - z) s for every k of two
+    groups, with a fractional zero point."""
+    N, K, gs = 96, 256, 128
+    case = W4Case(1, N, K, gs, 1, seed=31, zero_value=6.5)
+    qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, gs, 1, simt_cfg(32, 2, 1))
+    try:
+        for k in (0, 1, 4, 7, 8, 127, 128, 200, 255):
+            A = np.zeros((1, K), np.float16)
+            A[0, k] = 1.0
+            C = qg.qgemm_w4a16(to_dev(A), case.Wq, case.S, case.Z, group_size=gs)
+            ref = oracle.w4a16(A, case.Wq_host, case.h["scales"], case.h["zeros"], K, gs)
+            assert_fp16_close(C, ref, f"k={k}")
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, gs, 1, None)
+
+
+@pytest.mark.parametrize("rows,split_k", [(64, 2), (128, 1)])
+def test_w4a16_simt_full_size_sampled(rows, split_k):
+    N = K = 16384
+    case = W4Case(1, N, K, 128, 1, seed=rows)
+    qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, 128, 1, simt_cfg(rows, 4, split_k))
+    try:
+        C = case.run().float().cpu().numpy()
+    finally:
+        qg.qgemm_set_config(qg.OP_W4A16, 1, N, K, 128, 1, None)
+    ms, ns = sample_pairs(1, N, 2000, seed=rows)
+    assert_fp16_close(torch.from_numpy(C[ms, ns]), case.ref_at(ms, ns), "simt full size")
+
+
 def test_w4a16_one_hot_element_order():
     """A = e_k for every k of a 256-wide K: C[k, n] must be exactly fp16((q[n,k] - z) * s)."""
     N, K, gs = 48, 256, 64
