@@ -36,7 +36,8 @@ PATH_AUTO, PATH_GEMV, PATH_TC, PATH_STREAM = 0, 1, 2, 3
 # every symbol include/qgemm.h declares
 EXPORTS = (
     "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes",
-    "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w4a16_host", "qgemm_w4a16_host_workspace_bytes",
+    "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
     "quant_rtn_int4", "qgemm_w8a8_requant",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.qgemm_w8a8_requant.argtypes = [vp, vp, vp, vp, i32, i32, i32, vp]
         L.qgemm_w4a16_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
         L.qgemm_w4a16_workspace_bytes.restype = ctypes.c_size_t
+        L.qgemm_w4a16_host.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
+                                       ctypes.c_size_t, vp]
+        L.qgemm_w4a16_host_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.qgemm_w4a16_host_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_w2a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_dense_f16.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
@@ -102,7 +107,7 @@ def lib() -> ctypes.CDLL:
         L.qgemm_version.restype = i32
         for name in EXPORTS:
             if name not in ("qgemm_status_string", "qgemm_clear_configs", "qgemm_version",
-                            "qgemm_w4a16_workspace_bytes"):
+                            "qgemm_w4a16_workspace_bytes", "qgemm_w4a16_host_workspace_bytes"):
                 getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -236,6 +241,40 @@ def qgemm_w4a16_splitk_f32(A, Wq, scales, zeros=None, C=None, group_size: int = 
                                       _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "qgemm_w4a16_splitk_f32")
     return C
+
+
+def qgemm_w4a16_host_workspace_bytes(M: int, N: int, K: int, chunk_tokens: int = 0) -> int:
+    return int(lib().qgemm_w4a16_host_workspace_bytes(M, N, K, chunk_tokens))
+
+
+def qgemm_w4a16_host(A_host, Wq, scales, zeros, C_host, workspace, group_size: int = 128,
+                     split_k: int = 0, stream=None):
+    """W4A16 with A_host fp16 [M,K] and C_host fp16 [M,N] in page-locked host memory (CPU tensors
+    from pin_memory()); A streams in and C out in chunks through `workspace` (a uint8 CUDA tensor
+    of qgemm_w4a16_host_workspace_bytes(...) bytes or more). Asynchronous on `stream`: wait on
+    it before reading C_host."""
+    torch = _torch()
+    for name, t in (("A_host", A_host), ("C_host", C_host)):
+        if t.dtype != torch.float16 or t.dim() != 2 or t.device.type != "cpu" or \
+                not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 2-D float16 CPU tensor")
+        if not t.is_pinned():
+            raise ValueError(f"{name} must be in page-locked memory (pin_memory())")
+    _need(Wq, (torch.int32, torch.uint32), 2, "Wq")
+    _need(scales, torch.float16, 2, "scales")
+    if zeros is not None:
+        _need(zeros, torch.float16, 2, "zeros")
+    _need(workspace, torch.uint8, 1, "workspace")
+    M, K = A_host.shape
+    N = Wq.shape[0]
+    if tuple(C_host.shape) != (M, N):
+        raise ValueError("C_host must be [M, N]")
+    st = lib().qgemm_w4a16_host(A_host.data_ptr(), _ptr(Wq), _ptr(scales), _ptr(zeros),
+                                C_host.data_ptr(), M, N, K, group_size, split_k,
+                                int(zeros is not None), _ptr(workspace), workspace.numel(),
+                                _stream(stream))
+    _check(st, "qgemm_w4a16_host")
+    return C_host
 
 
 def qgemm_w8a8(A, W, C=None, split_k: int = 0, stream=None):

@@ -549,6 +549,45 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
 
 using namespace qg;
 
+namespace qg {
+namespace {
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t in = nullptr, out = nullptr;                 // host-to-device, device-to-host
+    cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;   // one call's chain of records and waits at a time (events are reused)
+
+bool pipe_init(HostPipe &hp)
+{
+    if (hp.ready) return true;
+    const unsigned ev = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, ev) == cudaSuccess;
+    for (int b = 0; b < 2 && ok; ++b)
+        ok = cudaEventCreateWithFlags(&hp.in_done[b], ev) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.comp_done[b], ev) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.out_done[b], ev) == cudaSuccess;
+    hp.ready = ok;
+    return ok;
+}
+
+bool page_locked(const void *p)
+{
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+} // namespace
+} // namespace qg
+
+using namespace qg;
+
 extern "C" {
 
 qg_status qgemm_w4a16(const void *A, const uint32_t *Wq, const void *scales, const void *zeros,
@@ -612,6 +651,95 @@ qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *
         return QG_ERR_CUDA;
     }
     if (launch_gemv_w4a16_tma(p, c, d->err_word, stream, parts, counters) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+// ---- host-buffer form: chunks of tokens through double buffers, copies on their own streams --
+
+size_t qgemm_w4a16_host_workspace_bytes(int M, int N, int K, int chunk_tokens)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || chunk_tokens < 0) return 0;
+    const size_t mc = chunk_tokens ? (size_t)std::min(chunk_tokens, M) : (size_t)std::min(M, 2048);
+    const size_t a = (mc * K * 2 + 255) / 256 * 256, c = (mc * N * 2 + 255) / 256 * 256;
+    return 2 * (a + c);
+}
+
+
+qg_status qgemm_w4a16_host(const void *A_host, const uint32_t *Wq, const void *scales,
+                           const void *zeros, void *C_host, int M, int N, int K, int group_size,
+                           int split_k, int has_zero, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream)
+{
+    qg_status s = check_shape(QG_OP_W4A16, M, N, K, group_size, has_zero, split_k);
+    if (s != QG_OK) return s;
+    if (!A_host || !C_host || !Wq || !scales || !workspace) return QG_ERR_INVALID_ARG;
+    if ((zeros != nullptr) != (has_zero != 0)) return QG_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(Wq, 16) || !aligned(scales, 2) ||
+        (zeros && !aligned(zeros, 2)))
+        return QG_ERR_ALIGNMENT;
+    // chunk: the largest multiple of 256 tokens (or all M) whose double buffers fit
+    const size_t per_token = 4 * ((size_t)K + (size_t)N);
+    long mc = (long)std::min<size_t>((size_t)M, workspace_bytes / per_token);
+    if (mc < M) mc = mc / 256 * 256;
+    while (mc > 0 && qgemm_w4a16_host_workspace_bytes(M, N, K, (int)mc) > workspace_bytes)
+        mc = mc > 256 ? mc - 256 : mc - 1;
+    if (mc <= 0) return QG_ERR_INVALID_ARG;
+    DeviceInfo *d = nullptr;
+    s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (!page_locked(A_host) || !page_locked(C_host)) return QG_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    const size_t a_bytes = ((size_t)mc * K * 2 + 255) / 256 * 256;
+    const size_t c_bytes = ((size_t)mc * N * 2 + 255) / 256 * 256;
+    char *ws = static_cast<char *>(workspace);
+    void *Ad[2] = {ws, ws + a_bytes};
+    void *Cd[2] = {ws + 2 * a_bytes, ws + 2 * a_bytes + c_bytes};
+    const char *Ah = static_cast<const char *>(A_host);
+    char *Ch = static_cast<char *>(C_host);
+
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    HostPipe &hp = g_pipe[dev];
+    if (!pipe_init(hp)) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    bool good = ok(cudaEventRecord(hp.start, stream)) && ok(cudaStreamWaitEvent(hp.in, hp.start, 0)) &&
+                ok(cudaStreamWaitEvent(hp.out, hp.start, 0));
+    const int chunks = (int)((M + mc - 1) / mc);
+    for (int c = 0; c < chunks && good; ++c) {
+        const int b = c & 1;
+        const int rows = (int)std::min<long>(mc, M - (long)c * mc);
+        const size_t r0 = (size_t)c * mc;
+        // A buffer b is free once the matmul of chunk c - 2 has finished reading it
+        if (c >= 2) good = ok(cudaStreamWaitEvent(hp.in, hp.comp_done[b], 0));
+        good = good && ok(cudaMemcpyAsync(Ad[b], Ah + r0 * K * 2, (size_t)rows * K * 2,
+                                          cudaMemcpyHostToDevice, hp.in)) &&
+               ok(cudaEventRecord(hp.in_done[b], hp.in)) &&
+               ok(cudaStreamWaitEvent(stream, hp.in_done[b], 0));
+        // C buffer b is free once the copy-out of chunk c - 2 has finished
+        if (good && c >= 2) good = ok(cudaStreamWaitEvent(stream, hp.out_done[b], 0));
+        if (!good) break;
+        s = matmul(QG_OP_W4A16, Ad[b], Wq, scales, zeros, Cd[b], rows, N, K, group_size, split_k,
+                   has_zero, stream);
+        if (s != QG_OK) return s;
+        good = ok(cudaEventRecord(hp.comp_done[b], stream)) &&
+               ok(cudaStreamWaitEvent(hp.out, hp.comp_done[b], 0)) &&
+               ok(cudaMemcpyAsync(Ch + r0 * N * 2, Cd[b], (size_t)rows * N * 2,
+                                  cudaMemcpyDeviceToHost, hp.out)) &&
+               ok(cudaEventRecord(hp.out_done[b], hp.out));
+    }
+    // work queued on `stream` later waits for every copy into C_host
+    for (int b = 0; b < std::min(chunks, 2) && good; ++b)
+        good = ok(cudaStreamWaitEvent(stream, hp.out_done[b], 0));
+    if (!good) {
         cudaGetLastError();
         return QG_ERR_CUDA;
     }

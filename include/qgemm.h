@@ -176,6 +176,33 @@ qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, cons
                                          cudaStream_t stream);
 
 /*
+ * W4A16 with the activations and the result in page-locked host memory: one end-to-end call for
+ * a caller whose tokens live on the host. A goes in and C comes out in chunks of tokens through
+ * `workspace`, so that the host-to-device copy of one chunk, the matmul of the one before and
+ * the device-to-host copy of the one before that run at the same time (the two directions use
+ * separate copy engines). Each chunk is computed as qgemm_w4a16 computes it.
+ *   A_host: fp16 [M, K] row-major; C_host: fp16 [M, N] row-major; both page-locked
+ *   (cudaHostAlloc or cudaHostRegister; pageable memory returns QG_ERR_INVALID_ARG).
+ *   Wq, scales, zeros, group_size, split_k, has_zero: as qgemm_w4a16 (device memory).
+ *   workspace: caller-owned device memory, 256-byte aligned, holding two A chunks and two C
+ *   chunks; chunk = the largest multiple of 256 tokens (or M) with 4 * chunk * (K + N) bytes
+ *   <= workspace_bytes; qgemm_w4a16_host_workspace_bytes gives the size for a chosen chunk.
+ * Stream order as for every call: the copies start after the work already queued on `stream`,
+ * and work queued on `stream` later starts after the last copy into C_host has finished (wait
+ * on `stream` before reading C_host on the host). The library creates two copy streams and a
+ * few events per device on first use (no device memory). Calls that share a workspace must be
+ * ordered on one stream. On an error return the contents of C_host are undefined.
+ */
+qg_status qgemm_w4a16_host(const void *A_host, const uint32_t *Wq, const void *scales,
+                           const void *zeros, void *C_host, int M, int N, int K, int group_size,
+                           int split_k, int has_zero, void *workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* Workspace bytes for qgemm_w4a16_host with chunks of chunk_tokens tokens (0: min(M, 2048));
+ * 0 if the arguments are invalid. */
+size_t qgemm_w4a16_host_workspace_bytes(int M, int N, int K, int chunk_tokens);
+
+/*
  * W8A8. A: int8 [M, K]. W: int8 [N, K]. C: int32 [M, N] = sum_k A[m,k] * W[n,k], exact
  * (it wraps modulo 2^32 only if |C| >= 2^31, impossible for K <= 131072).
  * group_size must be -1 or 0 (no scales) and has_zero 0. Requires K % 16 == 0.

@@ -259,3 +259,31 @@ def test_splitk_f32_validation_without_gpu():
         qg.QG_ERR_INVALID_ARG                                         # workspace too small
     assert L.qgemm_w4a16_splitk_f32(A, W, S, Z, C, 1, 64, 256, 128, 2, 1,
                                     ctypes.c_void_p(0x100010), need, None) == qg.QG_ERR_ALIGNMENT
+
+
+def test_host_workspace_bytes():
+    # two A chunks and two C chunks, each rounded up to 256 bytes
+    assert qg.qgemm_w4a16_host_workspace_bytes(16384, 16384, 16384, 2048) == \
+        2 * (2048 * 16384 * 2 + 2048 * 16384 * 2)
+    assert qg.qgemm_w4a16_host_workspace_bytes(1, 100, 64, 0) == 2 * (256 + 256)
+    assert qg.qgemm_w4a16_host_workspace_bytes(5000, 64, 64, 0) == \
+        qg.qgemm_w4a16_host_workspace_bytes(5000, 64, 64, 2048)
+    assert qg.qgemm_w4a16_host_workspace_bytes(0, 64, 64, 0) == 0
+
+
+def test_host_form_validation_without_gpu():
+    L = qg.lib()
+    ws = ctypes.c_void_p(0x100000)
+    need = qg.qgemm_w4a16_host_workspace_bytes(8, 64, 256, 0)
+    assert L.qgemm_w4a16_host(None, W, S, Z, C, 8, 64, 256, 128, 0, 1, ws, need, None) == \
+        qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 256, 128, 0, 1, None, need, None) == \
+        qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_w4a16_host(A, W, S, None, C, 8, 64, 256, 128, 0, 1, ws, need, None) == \
+        qg.QG_ERR_INVALID_ARG                                         # zeros vs has_zero
+    assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 256, 128, 0, 1, ws, 100, None) == \
+        qg.QG_ERR_INVALID_ARG                                         # no chunk fits
+    assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 256, 128, 0, 1, ctypes.c_void_p(0x100010),
+                              need, None) == qg.QG_ERR_ALIGNMENT
+    assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 100, 128, 0, 1, ws, need, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
