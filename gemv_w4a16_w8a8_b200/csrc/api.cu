@@ -713,11 +713,30 @@ qg_status qgemm_w4a16_host(const void *A_host, const uint32_t *Wq, const void *s
     auto ok = [](cudaError_t e) { return e == cudaSuccess; };
     bool good = ok(cudaEventRecord(hp.start, stream)) && ok(cudaStreamWaitEvent(hp.in, hp.start, 0)) &&
                 ok(cudaStreamWaitEvent(hp.out, hp.start, 0));
-    const int chunks = (int)((M + mc - 1) / mc);
+    // chunks: a quarter-size first and last chunk when there are more than two (the first
+    // copy in and the last copy out overlap nothing), full chunks between them
+    std::vector<std::pair<long, long>> sched;   // (first token, tokens)
+    {
+        const long q = std::max(256L, mc / 4 / 256 * 256);
+        const bool ramp = M > 2 * mc && q < mc;
+        const long tail = ramp ? q : 0;
+        long r = 0;
+        if (ramp) {
+            sched.push_back({0, q});
+            r = q;
+        }
+        while (r < M - tail) {
+            const long n = std::min(mc, M - tail - r);
+            sched.push_back({r, n});
+            r += n;
+        }
+        if (tail) sched.push_back({r, M - r});
+    }
+    const int chunks = (int)sched.size();
     for (int c = 0; c < chunks && good; ++c) {
         const int b = c & 1;
-        const int rows = (int)std::min<long>(mc, M - (long)c * mc);
-        const size_t r0 = (size_t)c * mc;
+        const int rows = (int)sched[c].second;
+        const size_t r0 = (size_t)sched[c].first;
         // A buffer b is free once the matmul of chunk c - 2 has finished reading it
         if (c >= 2) good = ok(cudaStreamWaitEvent(hp.in, hp.comp_done[b], 0));
         good = good && ok(cudaMemcpyAsync(Ad[b], Ah + r0 * K * 2, (size_t)rows * K * 2,

@@ -187,6 +187,8 @@ qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, cons
  *   workspace: caller-owned device memory, 256-byte aligned, holding two A chunks and two C
  *   chunks; chunk = the largest multiple of 256 tokens (or M) with 4 * chunk * (K + N) bytes
  *   <= workspace_bytes; qgemm_w4a16_host_workspace_bytes gives the size for a chosen chunk.
+ *   With more than two chunks the first and the last are a quarter of a chunk (at least 256
+ *   tokens): their copies are the ones nothing else overlaps.
  * Stream order as for every call: the copies start after the work already queued on `stream`,
  * and work queued on `stream` later starts after the last copy into C_host has finished (wait
  * on `stream` before reading C_host on the host). The library creates two copy streams and a

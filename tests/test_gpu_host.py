@@ -30,7 +30,9 @@ def host_case(M, N, K, gs, hz, seed):
                                                (700, 384, 1024, 128, 0, 0),     # one chunk
                                                (1, 4096, 4096, 128, 1, 0),
                                                (513, 136, 512, 64, 1, 256),
-                                               (1024, 520, 2048, 128, 1, 256)])
+                                               (1024, 520, 2048, 128, 1, 256),
+                                               # 256 + 1024 + 1024 + 440 + 256 (ramped ends)
+                                               (3000, 264, 512, 128, 1, 1024)])
 def test_host_form_matches_oracle(M, N, K, gs, hz, chunk):
     A_host, C_host, Wq, S, Z, ref = host_case(M, N, K, gs, bool(hz), seed=M + N)
     ws = torch.empty(qg.qgemm_w4a16_host_workspace_bytes(M, N, K, chunk), dtype=torch.uint8,
