@@ -53,6 +53,15 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "w4a16_nk16384"
 
 
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum):
+# the weight-major tile (256 tokens, 3 stages) on M = 2048, N = K = 16384 measured 605.2 MB read
+# + 60.9 MB written; an M = 16384 launch runs the same pattern (8 token tiles against all 128
+# weight tiles, weights read once per group) 8 times, so its traffic is scaled by 8.
+TRAFFIC_BYTES = {(16384, 16384, 16384): 8 * (605178368 + 60862208)}
+TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 2048 launch of the "
+                  "same tile, scaled by its 8 groups of token tiles")
+
+
 def shape_bytes(op, M, K, N, has_zero, gs=128):
     if op == "w4a16":
         return N * K // 2 + N * (K // gs) * 2 * (1 + has_zero) + 2 * M * K + 2 * M * N
@@ -328,7 +337,14 @@ def run_ours(args, world, rank, local):
         achieved = by / (ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
-    roof["traffic"] = args.traffic
+    if args.traffic is not None:
+        roof["traffic"] = args.traffic
+    elif (M, K, N) in TRAFFIC_BYTES and sp["cfg"]["path"] == 2 and sp["cfg"]["bn"] == 256 and \
+            sp["cfg"]["swap_ab"] == 1:
+        roof["traffic"] = TRAFFIC_BYTES[(M, K, N)]
+        roof["traffic_source"] = TRAFFIC_SOURCE
+    else:
+        roof["traffic"] = None
     roof["kernel_shape"] = [M, K, N]
     roof["peak_source"] = (f"{peaks['source']} "
                            f"({'burst' if timed_alone else 'sustained'} for tensor peaks)")
