@@ -49,7 +49,28 @@ WORKLOADS = {
     "w4a16_nk16384_small_m": {"op": "w4a16", "has_zero": 1,
                               "shapes": [(1, 16384, 16384), (32, 16384, 16384),
                                          (128, 16384, 16384)]},
+    # int8 x int8 -> int32 and int8 x int2 -> int32 over the BitBLAS M sweep at N = K = 16384
+    "w8a8_nk16384": {"op": "w8a8", "has_zero": 0,
+                     "shapes": [(1, 16384, 16384), (32, 16384, 16384), (128, 16384, 16384),
+                                (512, 16384, 16384)]},
+    "w2a8_nk16384": {"op": "w2a8", "has_zero": 0,
+                     "shapes": [(1, 16384, 16384), (32, 16384, 16384), (128, 16384, 16384),
+                                (512, 16384, 16384)]},
+    # the compute-bound shapes: W4A16 without zero points, and the dense fp16 baseline
+    "w4a16_nozero_large_m": {"op": "w4a16", "has_zero": 0,
+                             "shapes": [(512, 16384, 16384), (16384, 16384, 16384)]},
+    "dense_large_m": {"op": "dense", "has_zero": 0,
+                      "shapes": [(512, 16384, 16384), (16384, 16384, 16384)]},
 }
+METRICS = {
+    "w4a16": "int4-weight GEMM TFLOP/s & effective HBM GB/s, M=1..16384, N=K=16384",
+    "w8a8": "int8 x int8 -> int32 GEMM TOP/s & effective HBM GB/s, N=K=16384",
+    "w2a8": "int8 x int2 -> int32 GEMM TOP/s & effective HBM GB/s, N=K=16384",
+    "dense": "fp16 x fp16 -> fp16 GEMM TFLOP/s (in-library baseline), N=K=16384",
+}
+DTYPES = {"w4a16": "f16xu4->f32acc->f16", "w8a8": "s8xs8->s32", "w2a8": "s8xs2->s32",
+          "dense": "f16xf16->f32acc->f16"}
+UNITS = {"w4a16": "TFLOP/s", "w8a8": "TOP/s", "w2a8": "TOP/s", "dense": "TFLOP/s"}
 DEFAULT_WORKLOAD = "w4a16_nk16384"
 
 
@@ -185,6 +206,70 @@ def barrier(world: int, device=None):
 
 # ---- our arm ----------------------------------------------------------------------------------------
 
+def OP_CODES_table():
+    import gemv_w4a16_w8a8_b200 as qg
+    return {"w4a16": qg.OP_W4A16, "w8a8": qg.OP_W8A8, "w2a8": qg.OP_W2A8,
+            "dense": qg.OP_DENSE_F16}
+
+
+OP_CODES = {k: (lambda k=k: OP_CODES_table()[k]) for k in ("w4a16", "w8a8", "w2a8", "dense")}
+
+
+def prepare_shape(op, M, K, N, hz, gs, seed, dev):
+    """Seeded inputs of one shape in HBM (weights replicated into enough copies, >= 3x L2 in
+    total, that consecutive calls never find theirs in L2), plus page-locked host copies of A
+    and C for the end-to-end form."""
+    import torch
+    import gemv_w4a16_w8a8_b200 as qg
+    from gemv_w4a16_w8a8_b200 import synth
+    sp = {"M": M, "K": K, "N": N}
+    if op == "w4a16":
+        d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=seed)
+        A_np = d["A"]
+        codes = torch.from_numpy(d["codes"]).to(dev)
+        W0 = qg.quant_pack_int4(codes)
+        del codes
+        sp["S"] = torch.from_numpy(d["scales"]).to(dev)
+        sp["Z"] = torch.from_numpy(d["zeros"]).to(dev) if hz else None
+        c_dtype, wbytes = torch.float16, N * K // 2
+    elif op == "w8a8":
+        d = synth.w8a8_inputs(M, N, K, seed=seed)
+        A_np = d["A"]
+        W0 = torch.from_numpy(d["W"]).to(dev)
+        c_dtype, wbytes = torch.int32, N * K
+    elif op == "w2a8":
+        d = synth.w2a8_inputs(M, N, K, seed=seed)
+        A_np = d["A"]
+        W0 = qg.quant_pack_int2(torch.from_numpy(d["Wv"]).to(dev))
+        c_dtype, wbytes = torch.int32, N * K // 4
+    else:
+        d = synth.dense_inputs(M, N, K, seed=seed)
+        A_np = d["A"]
+        W0 = torch.from_numpy(d["W"]).to(dev)
+        c_dtype, wbytes = torch.float16, 2 * N * K
+    n_sets = max(1, min(64, math.ceil(3 * L2_BYTES / wbytes)))
+    sp.update({"A": torch.from_numpy(A_np).to(dev), "W": [W0] + [W0.clone() for _ in range(n_sets - 1)],
+               "C": torch.empty((M, N), dtype=c_dtype, device=dev), "n_sets": n_sets,
+               "A_host": torch.from_numpy(A_np).pin_memory(),
+               "C_host": torch.empty((M, N), dtype=c_dtype).pin_memory()})
+    return sp
+
+
+def matmul(op, sp, W, gs, A=None, C=None):
+    """One call of the library's entry point for this op."""
+    import gemv_w4a16_w8a8_b200 as qg
+    A = sp["A"] if A is None else A
+    C = sp["C"] if C is None else C
+    if op == "w4a16":
+        qg.qgemm_w4a16(A, W, sp["S"], sp["Z"], C=C, group_size=gs)
+    elif op == "w8a8":
+        qg.qgemm_w8a8(A, W, C=C)
+    elif op == "w2a8":
+        qg.qgemm_w2a8(A, W, C=C)
+    else:
+        qg.qgemm_dense_f16(A, W, C=C)
+
+
 def run_ours(args, world, rank, local):
     import torch
     import gemv_w4a16_w8a8_b200 as qg
@@ -204,34 +289,20 @@ def run_ours(args, world, rank, local):
 
     # inputs: one A per shape; weights: each shape's packed matrix replicated into enough
     # copies (>= 3x L2 in total) that consecutive calls of a shape never find theirs in L2
-    per_shape = []
-    for si, (M, K, N) in enumerate(shapes):
-        d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=1000 * si)
-        A = torch.from_numpy(d["A"]).to(dev)
-        codes = torch.from_numpy(d["codes"]).to(dev)
-        S = torch.from_numpy(d["scales"]).to(dev)
-        Z = torch.from_numpy(d["zeros"]).to(dev) if hz else None
-        Wq0 = qg.quant_pack_int4(codes)
-        del codes
-        n_sets = max(1, min(64, math.ceil(3 * L2_BYTES / (N * K // 2))))
-        sets = [Wq0] + [Wq0.clone() for _ in range(n_sets - 1)]
-        C = torch.empty((M, N), dtype=torch.float16, device=dev)
-        per_shape.append({"M": M, "K": K, "N": N, "A": A, "S": S, "Z": Z, "W": sets, "C": C,
-                          "n_sets": n_sets,
-                          "A_host": torch.from_numpy(d["A"]).pin_memory(),
-                          "C_host": torch.empty((M, N), dtype=torch.float16).pin_memory()})
-        del d
+    per_shape = [prepare_shape(op, M, K, N, hz, gs, 1000 * si, dev)
+                 for si, (M, K, N) in enumerate(shapes)]
     torch.cuda.synchronize()
 
     # configuration search (once per shape, before timing)
     tuned = []
     for sp in per_shape:
         M, K, N = sp["M"], sp["K"], sp["N"]
+        g_op = gs if op == "w4a16" else -1
         if args.no_tune:
-            cfg = qg.qgemm_plan(qg.OP_W4A16, M, N, K, gs, hz)
+            cfg = qg.qgemm_plan(OP_CODES[op](), M, N, K, g_op, hz)
         else:
-            cfg = qg.qgemm_tune(qg.OP_W4A16, sp["A"], sp["W"][0], sp["S"], sp["Z"], sp["C"],
-                                M, N, K, gs, hz, reps=args.tune_reps)
+            cfg = qg.qgemm_tune(OP_CODES[op](), sp["A"], sp["W"][0], sp.get("S"), sp.get("Z"),
+                                sp["C"], M, N, K, g_op, hz, reps=args.tune_reps)
         sp["cfg"] = cfg
         tuned.append({"shape": [M, K, N], **{k: cfg[k] for k in ("path", "rows", "bm", "bn",
                                                                    "bk", "stages", "split_k")}})
@@ -240,8 +311,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
 
     def call(sp, i):
-        qg.qgemm_w4a16(sp["A"], sp["W"][i % sp["n_sets"]], sp["S"], sp["Z"], C=sp["C"],
-                       group_size=gs)
+        matmul(op, sp, sp["W"][i % sp["n_sets"]], gs)
 
     n_sets = max(sp["n_sets"] for sp in per_shape)
 
@@ -316,7 +386,7 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
 
     # ---- end to end: host A in, host C out, through the same entry point ----
-    e2e = run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step)
+    e2e = run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step)
 
     # ---- roofline of the dominant call ----
     j = int(np.argmax(shape_ms))
@@ -327,12 +397,14 @@ def run_ours(args, world, rank, local):
     ms = shape_ms[j]
     intensity = fl / by
     timed_alone = total_ms < 1000.0
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)   # flop per byte
+    # int8 contractions: the measured bf16 peak times the nominal dense int8 / bf16 ratio (2)
+    tscale = 2.0 if op in ("w8a8", "w2a8") else 1.0
+    tpeak = tscale * (peaks["bf16_tflops"] if timed_alone else peaks["bf16_tflops_sustained"])
+    ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)   # flop per byte
     if intensity >= ridge:
-        peak = peaks["bf16_tflops"] if timed_alone else peaks["bf16_tflops_sustained"]
         achieved = fl / (ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(tpeak, 1),
+                "unit": UNITS[op], "frac": round(achieved / tpeak, 4)}
     else:
         achieved = by / (ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
@@ -347,7 +419,9 @@ def run_ours(args, world, rank, local):
         roof["traffic"] = None
     roof["kernel_shape"] = [M, K, N]
     roof["peak_source"] = (f"{peaks['source']} "
-                           f"({'burst' if timed_alone else 'sustained'} for tensor peaks)")
+                           f"({'burst' if timed_alone else 'sustained'} for tensor peaks"
+                           + (", x2 for int8 (nominal dense int8 / bf16)" if tscale != 1 else "")
+                           + ")")
 
     details = []
     for s, t in zip(per_shape, shape_ms):
@@ -359,9 +433,9 @@ def run_ours(args, world, rank, local):
                         "hbm_frac": round(by_s / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
 
     out = {
-        "metric": "int4-weight GEMM TFLOP/s & effective HBM GB/s, M=1..16384, N=K=16384",
+        "metric": METRICS[op],
         "value": round(value, 3),
-        "unit": "TFLOP/s",
+        "unit": UNITS[op],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": warm_steps,
@@ -369,7 +443,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16xu4->f32acc->f16",
+        "dtype": DTYPES[op],
         "data": "synthetic",
         "config": {"workload": args.workload, "op": op, "shapes_mkn": [list(s) for s in shapes],
                    "group_size": gs, "has_zero": hz, "parallelism": f"replicas{world}",
@@ -394,24 +468,31 @@ def run_ours(args, world, rank, local):
     return out
 
 
-def run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step):
-    """The same step end to end through the host-buffer entry point: A from page-locked host
-    memory in, C to page-locked host memory out, every shape every step. The call streams
-    chunks of tokens through a device workspace so that both copy directions overlap the
-    matmul."""
+def run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step):
+    """The same step end to end: A from page-locked host memory in, C to page-locked host
+    memory out, every shape every step. W4A16 goes through the host-buffer entry point, which
+    streams chunks of tokens through a device workspace so that both copy directions overlap
+    the matmul; the other ops copy A in, call, and copy C out on the stream."""
     import torch
     import gemv_w4a16_w8a8_b200 as qg
     steps = max(1, min(args.steps, 5))
-    h2d = sum(sp["A_host"].numel() * 2 for sp in per_shape)
-    d2h = sum(sp["C_host"].numel() * 2 for sp in per_shape)
-    ws_bytes = max(qg.qgemm_w4a16_host_workspace_bytes(sp["M"], sp["N"], sp["K"], 0)
-                   for sp in per_shape)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    h2d = sum(sp["A_host"].numel() * sp["A_host"].element_size() for sp in per_shape)
+    d2h = sum(sp["C_host"].numel() * sp["C_host"].element_size() for sp in per_shape)
+    if op == "w4a16":
+        ws_bytes = max(qg.qgemm_w4a16_host_workspace_bytes(sp["M"], sp["N"], sp["K"], 0)
+                       for sp in per_shape)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
     def one(i):
         for sp in per_shape:
-            qg.qgemm_w4a16_host(sp["A_host"], sp["W"][i % len(sp["W"])], sp["S"], sp["Z"],
-                                sp["C_host"], ws, group_size=gs)
+            W = sp["W"][i % len(sp["W"])]
+            if op == "w4a16":
+                qg.qgemm_w4a16_host(sp["A_host"], W, sp["S"], sp["Z"], sp["C_host"], ws,
+                                    group_size=gs)
+            else:
+                sp["A"].copy_(sp["A_host"], non_blocking=True)
+                matmul(op, sp, W, gs)
+                sp["C_host"].copy_(sp["C"], non_blocking=True)
 
     one(0)
     torch.cuda.synchronize()
@@ -425,11 +506,12 @@ def run_e2e(args, per_shape, gs, hz, stream, world, dev, flops_step):
     e1.record(stream)
     torch.cuda.synchronize()
     value, ms = job_throughput(e0.elapsed_time(e1), flops_step, steps, world, dev)
-    return {"value": round(value, 3), "unit": "TFLOP/s",
+    path = ("qgemm_w4a16_host (pinned host A and C, chunks of up to 2048 tokens, copies in both "
+            "directions overlapped with the matmul)" if op == "w4a16" else
+            "pinned host A copied in, the call, C copied out, on one stream")
+    return {"value": round(value, 3), "unit": UNITS[op],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3),
-            "path": "qgemm_w4a16_host (pinned host A and C, chunks of up to 2048 tokens, copies "
-                    "in both directions overlapped with the matmul)"}
+            "ms_per_step": round(ms / steps, 3), "path": path}
 
 
 # ---- oracle arm ------------------------------------------------------------------------------------
@@ -449,21 +531,43 @@ def oracle_sample_rates(workload: str, budget_s: float, seed: int = 0):
     threads = oracle.max_threads()
     per = budget_s / len(wl["shapes"])
     out = []
+    op = wl["op"]
     for si, (M, K, N) in enumerate(wl["shapes"]):
         m_s = min(M, 256)
-        key = (m_s, min(N, 8192), K, hz, seed + si)
+        n_all = min(N, 8192)
+        key = (op, m_s, n_all, K, hz, seed + si)
         if key not in _ORACLE_INPUTS:
-            d = synth.w4a16_inputs(m_s, min(N, 8192), K, gs, bool(hz), seed=seed + si)
-            _ORACLE_INPUTS[key] = (d, oracle.pack_int4(d["codes"]))
-        d, Wq_all = _ORACLE_INPUTS[key]
+            if op == "w4a16":
+                d = synth.w4a16_inputs(m_s, n_all, K, gs, bool(hz), seed=seed + si)
+                d["Wq"] = oracle.pack_int4(d["codes"])
+            elif op == "w8a8":
+                d = synth.w8a8_inputs(m_s, n_all, K, seed=seed + si)
+            elif op == "w2a8":
+                d = synth.w2a8_inputs(m_s, n_all, K, seed=seed + si)
+                d["Wq"] = oracle.pack_int2(d["Wv"])
+            else:
+                d = synth.dense_inputs(m_s, n_all, K, seed=seed + si)
+            _ORACLE_INPUTS[key] = d
+        d = _ORACLE_INPUTS[key]
+
+        def run_slice(n):
+            if op == "w4a16":
+                oracle.w4a16(d["A"], d["Wq"][:n], d["scales"][:n],
+                             None if d["zeros"] is None else d["zeros"][:n], K, gs, nthreads=threads)
+            elif op == "w8a8":
+                oracle.w8a8(d["A"], d["W"][:n], nthreads=threads)
+            elif op == "w2a8":
+                oracle.w2a8(d["A"], d["Wq"][:n], nthreads=threads)
+            else:
+                oracle.dense_f16(d["A"], d["W"][:n], nthreads=threads)
+
         n_s, dt = 8, 0.0
         for _ in range(8):
-            n_s = min(n_s, Wq_all.shape[0])
+            n_s = min(n_s, n_all)
             t = time.perf_counter()
-            oracle.w4a16(d["A"], Wq_all[:n_s], d["scales"][:n_s],
-                         None if d["zeros"] is None else d["zeros"][:n_s], K, gs, nthreads=threads)
+            run_slice(n_s)
             dt = time.perf_counter() - t
-            if dt >= 0.5 * per or n_s >= Wq_all.shape[0]:
+            if dt >= 0.5 * per or n_s >= n_all:
                 break
             n_s = int(n_s * min(16.0, max(2.0, 0.9 * per / max(dt, 1e-6))))
         out.append((2.0 * m_s * n_s * K, dt, f"{m_s}x{n_s} of ({M},{K},{N})"))
@@ -476,7 +580,7 @@ def cpu_baseline(workload: str, budget_s: float = 15.0):
     # time the oracle would take for the whole step, shape by shape at its sampled rate
     est_s = sum(shape_flops(M, K, N) / (f / t) for (M, K, N), (f, t, _) in zip(wl["shapes"], rates))
     total = sum(shape_flops(M, K, N) for M, K, N in wl["shapes"])
-    return {"value": total / est_s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+    return {"value": total / est_s / 1e12, "unit": UNITS[wl["op"]], "cores": threads, "kind": "oracle",
             "sample": "; ".join(desc for _, _, desc in rates) +
                       f" (fp64 oracle, {sum(t for _, t, _ in rates):.1f} s wall on {threads} threads; "
                       f"each shape's rate applied to its full FLOPs)"}
@@ -502,17 +606,17 @@ def run_reference(args, world, rank):
     value = total_flops / (ms_per_step * 1e-3) / 1e12
     return {
         "impl": "reference",
-        "metric": "int4-weight GEMM TFLOP/s & effective HBM GB/s, M=1..16384, N=K=16384",
-        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRICS[wl["op"]],
+        "value": value, "unit": UNITS[wl["op"]], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "op": wl["op"],
                    "shapes_mkn": [list(s) for s in wl["shapes"]], "group_size": 128,
                    "has_zero": wl["has_zero"], "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNITS[wl["op"]], "cores": threads, "kind": "oracle",
                          "sample": samples + " per step; each shape's sampled rate applied to "
                                              "its full FLOPs"},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": value, "unit": UNITS[wl["op"]], "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
 
