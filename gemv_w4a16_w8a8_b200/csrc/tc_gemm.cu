@@ -1,21 +1,29 @@
-// tcgen05 tensor-core GEMM family for the compute-bound regime (M from a few dozen tokens up).
+// tcgen05 tensor-core GEMM family (dense fp16, W8A8, W4A16, W2A8): tcgen05.mma with operands in
+// shared memory and the accumulator in TMEM, fed by TMA, one persistent CTA of 512 threads per
+// SM walking work units (weight tile, token tile, K part).
 //
-//   D[128 weight rows, BN tokens] = W_tile[128, K] . A_tile[BN, K]^T     (both K-contiguous)
+// Two tile orientations, because an MMA from shared memory at M = 128 occupies the tensor pipe
+// ~98 cycles for any N up to 128 and reaches its full rate only at N = 256 (measured):
+//   weight-major   D[128 weight rows, BN tokens] = W_tile . A_tile^T, BN in {16..256}; the
+//                  large-M tile (BN = 256) upcasts each weight once per 256 tokens;
+//   token-major    D[128 tokens, 256 weight rows] = A_tile . W_tile^T (W4A16): tokens are the A
+//                  operand (rows past M read as zero), 256 upcast weight rows the B operand, so
+//                  every MMA runs at N = 256 for 1..128 tokens.
 //
-// The weights fill the MMA's 128-row M side and the tokens its N side (16..256), so the per-FLOP
-// cost of dequantising weights falls as the token tile grows. One CTA (256 threads) per output
-// tile, warp-specialised:
-//   warp 0      TMA producer: a ring of `STAGES` shared-memory stages, each holding one 128-byte
-//               wide k-slab of the weight tile and of the activation tile (SWIZZLE_128B), tracked
-//               by mbarriers with transaction counts (multi-stage software pipelining, hidet-org/
-//               hidet issue #364; the stage count is a tunable, as the issue's num_stages);
-//   warp 1      allocates the TMEM accumulator, issues tcgen05.mma (kind::f16 for fp16 operands,
-//               kind::i8 for int8 operands) from one thread and commits each stage back to the
-//               producer;
-//   warps 4-7   for packed weights, upcast the packed slab to fp16 / int8 directly into the
-//               canonical K-major SWIZZLE_128B layout the MMA reads (LOP3 magic-number upcast,
-//               PRMT re-ordering); then, for every mode, the epilogue: tcgen05.ld of the fp32 /
-//               int32 accumulator, conversion, and a store or, for split-K, red.global.add.
+// Roles (warp-specialised):
+//   warp 4      TMA producer of the activation ring (and the weight slab for fp16 / int8
+//               weights): STAGES 128-byte-wide K slabs under SWIZZLE_128B, mbarrier transaction
+//               counts (multi-stage software pipelining with a tunable stage count, as the
+//               num_stages search in hidet-org/hidet issue #364);
+//   warp 6      TMA producer of the packed-weight ring (4-slab copies: 128 contiguous bytes of
+//               each weight row);
+//   warp 5      TMEM allocation and the MMA issue, one slab at a time, each slab's buffers
+//               committed back to their producers as soon as its MMAs complete;
+//   warps 8-15  upcast of packed weights into the K-major SWIZZLE_128B layout the MMA reads
+//               (LOP3 magic-number upcast, PRMT re-ordering, HFMA2 with the group's scale and
+//               zero), handed over per slab or per copy;
+//   warps 0-3   epilogue: tcgen05.ld of the double-buffered accumulator, conversion, stores or
+//               red.global.add for split-K (parallel-k through atomics, hidet issue #364).
 // Every wait is bounded (%globaltimer); a wait that runs out raises the device error word, makes
 // the other roles stop, lets in-flight copies land, frees TMEM and returns.
 #include <cuda.h>

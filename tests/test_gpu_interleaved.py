@@ -20,9 +20,11 @@ def test_pack_int4_interleaved_bit_exact():
         assert np.array_equal(got, oracle.pack_int4_interleaved(codes)), (N, K)
 
 
-def _cfg(path, rows=0, bn=0, stages=0, split=1):
+def _cfg(path, rows=0, bn=0, stages=0, split=1, swap=None):
+    if swap is None:
+        swap = 1 if path == qg.PATH_TC else 0
     return {"path": path, "rows": rows, "bm": 128 if path == qg.PATH_TC else 0, "bn": bn,
-            "bk": 0, "stages": stages, "split_k": split, "swap_ab": 1 if path == qg.PATH_TC else 0}
+            "bk": 0, "stages": stages, "split_k": split, "swap_ab": swap}
 
 
 CONFIGS = [
@@ -32,10 +34,12 @@ CONFIGS = [
     _cfg(qg.PATH_GEMV, rows=16, stages=2, split=4),
     _cfg(qg.PATH_TC, bn=64, stages=3, split=1),           # tensor-core kernel
     _cfg(qg.PATH_TC, bn=256, stages=4, split=2),
+    _cfg(qg.PATH_TC, bn=256, stages=4, split=1, swap=0),  # token-major tile
+    _cfg(qg.PATH_TC, bn=256, stages=2, split=3, swap=0),
 ]
 
 
-@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: f"p{c['path']}r{c['rows']}b{c['bn']}s{c['stages']}k{c['split_k']}")
+@pytest.mark.parametrize("cfg", CONFIGS, ids=lambda c: f"p{c['path']}r{c['rows']}b{c['bn']}s{c['stages']}k{c['split_k']}w{c['swap_ab']}")
 @pytest.mark.parametrize("M,N,K,gs,hz", [(1, 200, 1024, 128, 1), (7, 136, 2048, 128, 0),
                                          (40, 256, 512, 128, 1), (3, 96, 512, 64, 1)])
 def test_w4a16_interleaved_paths(cfg, M, N, K, gs, hz):
