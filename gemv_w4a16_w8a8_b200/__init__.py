@@ -40,7 +40,8 @@ EXPORTS = (
     "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
     "quant_rtn_int4", "qgemm_w8a8_requant",
     "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
-    "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_status_string",
+    "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_selftest_bounded_wait",
+    "qgemm_status_string",
     "qgemm_version",
 )
 
@@ -102,6 +103,7 @@ def lib() -> ctypes.CDLL:
         L.qgemm_clear_configs.argtypes = []
         L.qgemm_clear_configs.restype = None
         L.qgemm_sync_check.argtypes = [vp]
+        L.qgemm_selftest_bounded_wait.argtypes = [i32, vp]
         L.qgemm_status_string.argtypes = [i32]
         L.qgemm_status_string.restype = ctypes.c_char_p
         L.qgemm_version.restype = i32
@@ -427,6 +429,13 @@ def qgemm_clear_configs():
 
 def qgemm_sync_check(stream=None):
     _check(lib().qgemm_sync_check(_stream(stream)), "qgemm_sync_check")
+
+
+def qgemm_selftest_bounded_wait(limit_us: int = 20000, stream=None):
+    """Queue a kernel whose bounded wait runs out after limit_us; the next qgemm_sync_check raises
+    QG_ERR_DEVICE_TIMEOUT."""
+    _check(lib().qgemm_selftest_bounded_wait(limit_us, _stream(stream)),
+           "qgemm_selftest_bounded_wait")
 
 
 def qgemm_version() -> int:

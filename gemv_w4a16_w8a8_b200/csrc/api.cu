@@ -1080,6 +1080,20 @@ void qgemm_clear_configs(void)
     g_pinned.clear();
 }
 
+qg_status qgemm_selftest_bounded_wait(int limit_us, cudaStream_t stream)
+{
+    if (limit_us < 1 || limit_us > 2000000) return QG_ERR_INVALID_ARG;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_wait_selftest(d->err_word, 1000ull * (unsigned long long)limit_us, stream) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 qg_status qgemm_sync_check(cudaStream_t stream)
 {
     DeviceInfo *d = nullptr;

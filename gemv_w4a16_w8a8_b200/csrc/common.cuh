@@ -50,6 +50,9 @@ cudaError_t launch_gemv_w4a16_stream(const Problem &p, const qgemm_config_t &cfg
 cudaError_t launch_gemv_w2a8_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
                                  cudaStream_t stream);
 cudaError_t launch_gemv_int(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
+// A kernel whose bounded wait can never be satisfied: it gives up after limit_ns and raises *err.
+cudaError_t launch_wait_selftest(unsigned int *err, unsigned long long limit_ns,
+                                 cudaStream_t stream);
 cudaError_t launch_pack_int4(const uint8_t *codes, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
 cudaError_t launch_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, int N, int K,

@@ -71,7 +71,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // try_wait, reads the clock and the abort flag only every 64 tries (the clock read goes to a
 // shared pipe), and backs off with nanosleep once the wait runs long.
 __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned int *err)
+                                       unsigned int *err, uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = 0;
@@ -82,7 +82,7 @@ __device__ __noinline__ inline bool mbar_wait(uint32_t bar, uint32_t parity, vol
             const uint64_t now = global_ns();
             if (t0 == 0) {
                 t0 = now;
-            } else if (now - t0 > kWaitLimitNs) {
+            } else if (now - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (err) atomicOr(err, 1u);
                 return false;

@@ -325,6 +325,15 @@ void qgemm_clear_configs(void);
  */
 qg_status qgemm_sync_check(cudaStream_t stream);
 
+/*
+ * Self-test of the failure path (no counterpart in the pages): queues on `stream` a kernel whose
+ * bounded mbarrier wait can never be satisfied. The wait gives up after limit_us microseconds
+ * (1 .. 2000000), raises the device error word exactly as a stalled matmul pipeline would, and the
+ * kernel returns: no trap, no fault, the context stays usable. The next qgemm_sync_check reports
+ * QG_ERR_DEVICE_TIMEOUT and clears the word.
+ */
+qg_status qgemm_selftest_bounded_wait(int limit_us, cudaStream_t stream);
+
 const char *qgemm_status_string(qg_status status);
 
 /* Library version as major * 10000 + minor * 100 + patch. */

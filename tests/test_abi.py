@@ -287,3 +287,9 @@ def test_host_form_validation_without_gpu():
                               need, None) == qg.QG_ERR_ALIGNMENT
     assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 100, 128, 0, 1, ws, need, None) == \
         qg.QG_ERR_UNSUPPORTED_SHAPE
+
+
+def test_selftest_limit_validated_before_the_device():
+    L = qg.lib()
+    assert L.qgemm_selftest_bounded_wait(0, None) == qg.QG_ERR_INVALID_ARG
+    assert L.qgemm_selftest_bounded_wait(2000001, None) == qg.QG_ERR_INVALID_ARG
