@@ -683,7 +683,7 @@ qg_status qgemm_w4a16_host(const void *A_host, const uint32_t *Wq, const void *s
     // chunk: the largest multiple of 256 tokens (or all M) whose double buffers fit
     const size_t per_token = 4 * ((size_t)K + (size_t)N);
     long mc = (long)std::min<size_t>((size_t)M, workspace_bytes / per_token);
-    if (mc < M) mc = mc / 256 * 256;
+    if (mc < M && mc >= 256) mc = mc / 256 * 256;   // whole 256-token tiles when there is room
     while (mc > 0 && qgemm_w4a16_host_workspace_bytes(M, N, K, (int)mc) > workspace_bytes)
         mc = mc > 256 ? mc - 256 : mc - 1;
     if (mc <= 0) return QG_ERR_INVALID_ARG;

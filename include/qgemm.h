@@ -185,8 +185,9 @@ qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, cons
  *   (cudaHostAlloc or cudaHostRegister; pageable memory returns QG_ERR_INVALID_ARG).
  *   Wq, scales, zeros, group_size, split_k, has_zero: as qgemm_w4a16 (device memory).
  *   workspace: caller-owned device memory, 256-byte aligned, holding two A chunks and two C
- *   chunks; chunk = the largest multiple of 256 tokens (or M) with 4 * chunk * (K + N) bytes
- *   <= workspace_bytes; qgemm_w4a16_host_workspace_bytes gives the size for a chosen chunk.
+ *   chunks; chunk = the largest multiple of 256 tokens (or M, or fewer than 256 tokens when
+ *   that is all that fits) with 4 * chunk * (K + N) bytes <= workspace_bytes (plus rounding of
+ *   each buffer to 256 bytes); qgemm_w4a16_host_workspace_bytes gives the size for a chunk.
  *   With more than two chunks the first and the last are a quarter of a chunk (at least 256
  *   tokens): their copies are the ones nothing else overlaps.
  * Stream order as for every call: the copies start after the work already queued on `stream`,

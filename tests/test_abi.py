@@ -287,6 +287,17 @@ def test_host_form_validation_without_gpu():
                               need, None) == qg.QG_ERR_ALIGNMENT
     assert L.qgemm_w4a16_host(A, W, S, Z, C, 8, 64, 100, 128, 0, 1, ws, need, None) == \
         qg.QG_ERR_UNSUPPORTED_SHAPE
+    # a workspace for fewer than 256 tokens still gives a usable (smaller) chunk: the call gets
+    # past validation to the device probe, which refuses without a GPU
+    small = qg.qgemm_w4a16_host_workspace_bytes(1000, 64, 256, 100)
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except ImportError:
+        has_gpu = False
+    if not has_gpu:
+        assert L.qgemm_w4a16_host(A, W, S, Z, C, 1000, 64, 256, 128, 0, 1, ws, small, None) in \
+            (qg.QG_ERR_CUDA, qg.QG_ERR_NOT_SM100)
 
 
 def test_selftest_limit_validated_before_the_device():
