@@ -72,3 +72,28 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_int_workload_and_non_zero_ranks():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0", "--workload", "w2a8_nk16384",
+                        "--cpu-budget", "4"],
+                       capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.strip()][-1])
+    assert d["unit"] == "TOP/s" and d["dtype"] == "f64" and d["config"]["op"] == "w2a8"
+    # under torchrun only rank 0 times the oracle; the others exit 0 without output
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_every_workload_is_consistent():
+    for name, wl in bench.WORKLOADS.items():
+        assert wl["op"] in bench.METRICS and wl["op"] in bench.UNITS and wl["op"] in bench.DTYPES
+        for M, K, N in wl["shapes"]:
+            assert bench.shape_bytes(wl["op"], M, K, N, wl["has_zero"]) > 0
+            assert bench.shape_flops(M, K, N) == 2.0 * M * N * K
