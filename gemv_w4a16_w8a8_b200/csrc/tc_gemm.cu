@@ -122,8 +122,9 @@ template <int MODE> struct Traits {
 //   dense / int8 weights: one ring of STAGES stages, each a weight slab and an activation slab
 //     loaded by TMA (SWIZZLE_128B) and read by the MMA.
 //   packed weights: three rings, so that no latency of one step sits in the cycle of another:
-//     STAGES activation slabs (TMA -> MMA), kPackedStages packed weight slabs (TMA -> upcast;
-//     4 KB each, so the upcast can run far ahead) and DQ upcast weight slabs (upcast -> MMA).
+//     STAGES activation slabs (TMA -> MMA), sp packed-weight copies of PG slabs each (TMA ->
+//     upcast, so the upcast can run far ahead; see packed_stages) and DQ upcast weight slabs
+//     (upcast -> MMA; see dq_buffers).
 constexpr int kMaxSmem = 227 * 1024;
 
 // Packed weights move PG slabs per copy: PG = 4 reads 128 contiguous bytes of each weight row
@@ -642,8 +643,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     settle(ahead);
                 }
             };
-            // PG slabs (one packed copy) per pass: the PG upcasts are independent, so their
-            // latencies overlap; one proxy fence covers all of them
+            // one packed copy (PG slabs) per iteration: the copy's loads are issued together, its
+            // slabs upcast one after another, each into the next free upcast buffer
             int it = 0;
             while (cur.u < units) {
                 uint32_t sc2[PG], nz2[PG];
