@@ -1,12 +1,27 @@
 """Benchmark of the low-bit matmul library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--no-extras]
 
 A step is one pass of the hot path over one batch of seeded synthetic input: for every shape
 of the workload one matmul call (argument checks, configuration lookup, split-K zeroing when
 the configuration splits K, the kernel). The per-shape configuration search runs once before
 the timed region, as a deployment would run it once per shape. Inputs sit in HBM before the
 timed region; weight sets rotate so that no call finds its weights in L2.
+
+After the timed region the device error word is checked (a kernel that gave up a bounded wait
+fails the run) and the output of every timed shape, under the configuration that was timed, is
+compared with the host oracle on sampled elements: one random element in every 128 x 128 tile
+of C plus its corners ("parity" in the line). Integer outputs must match exactly, fp16 outputs
+within |C - ref| <= 0.02 + 0.01 |ref| per element and 5e-3 relative Frobenius error over the
+sample. A failed check still prints the line and exits with status 3.
+
+The headline workload (--workload, default the N = K = 16384 W4A16 sweep over M) gives `value`.
+Unless --no-extras, the other benchmark configurations are timed after it, shape by shape, into
+"configs" of the same line: one-token W4A16 at K = N = 4096 with split_k 1 and 4, the LLaMA-style
+shapes with and without zero points, W8A8 and W2A8 over M at N = K = 16384, W4A16 without zero
+points and the dense fp16 baseline at M = 512 / 16384, and a sweep of the tensor-core pipeline
+depth (stages 2..5) on the large-M shapes.
 
 Prints one JSON line (rank 0). Under torchrun every rank runs the same workload on its own GPU
 (independent replicas, no collective on the data path); `value` is the whole-job throughput
@@ -32,6 +47,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 L2_BYTES = 126 * 1024 * 1024
+GS = 128
 
 # ---- workloads -------------------------------------------------------------------------------
 # Each shape: (M, K, N). W4A16: group_size 128, fp16 zeros fixed at 8 (has_zero=1) unless noted.
@@ -40,11 +56,17 @@ WORKLOADS = {
     "w4a16_nk16384": {"op": "w4a16", "has_zero": 1,
                       "shapes": [(1, 16384, 16384), (32, 16384, 16384), (128, 16384, 16384),
                                  (512, 16384, 16384), (16384, 16384, 16384)]},
+    # one token at K = N = 4096 (hidet issue #364, k-parts 1 and 4 sweep)
+    "w4a16_m1_k4096": {"op": "w4a16", "has_zero": 1, "shapes": [(1, 4096, 4096)]},
     # LLaMA-style layer shapes (hidet issue #364, k-parts=4 table), M = 1 and 128
     "w4a16_llama": {"op": "w4a16", "has_zero": 1,
                     "shapes": [(1, 4096, 11008), (1, 11008, 4096), (1, 4096, 4096),
                                (1, 4096, 32000), (128, 4096, 11008), (128, 11008, 4096),
                                (128, 4096, 4096), (128, 4096, 32000)]},
+    "w4a16_llama_nozero": {"op": "w4a16", "has_zero": 0,
+                           "shapes": [(1, 4096, 11008), (1, 11008, 4096), (1, 4096, 4096),
+                                      (1, 4096, 32000), (128, 4096, 11008), (128, 11008, 4096),
+                                      (128, 4096, 4096), (128, 4096, 32000)]},
     # the small-M part of the sweep alone
     "w4a16_nk16384_small_m": {"op": "w4a16", "has_zero": 1,
                               "shapes": [(1, 16384, 16384), (32, 16384, 16384),
@@ -73,6 +95,19 @@ DTYPES = {"w4a16": "f16xu4->f32acc->f16", "w8a8": "s8xs8->s32", "w2a8": "s8xs2->
 UNITS = {"w4a16": "TFLOP/s", "w8a8": "TOP/s", "w2a8": "TOP/s", "dense": "TFLOP/s"}
 DEFAULT_WORKLOAD = "w4a16_nk16384"
 
+# The other benchmark configurations, timed after the headline: (name, workload, explicit
+# split_k values timed on the planner's path before the search, stage sweep on the large shapes)
+EXTRAS = [
+    ("w4a16_m1_k4096_n4096", "w4a16_m1_k4096", (1, 4), False),
+    ("w4a16_llama", "w4a16_llama", (), False),
+    ("w4a16_llama_nozero", "w4a16_llama_nozero", (), False),
+    ("w8a8_nk16384", "w8a8_nk16384", (1, 4), False),
+    ("w2a8_nk16384", "w2a8_nk16384", (), False),
+    ("w4a16_nozero_large_m", "w4a16_nozero_large_m", (), True),
+    ("dense_large_m", "dense_large_m", (), True),
+]
+SWEEP_STAGES = (2, 3, 4, 5)
+
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum):
 # the weight-major tile (256 tokens, 3 stages) on M = 2048, N = K = 16384 measured 605.2 MB read
@@ -83,7 +118,7 @@ TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 2
                   "same tile, scaled by its 8 groups of token tiles")
 
 
-def shape_bytes(op, M, K, N, has_zero, gs=128):
+def shape_bytes(op, M, K, N, has_zero, gs=GS):
     if op == "w4a16":
         return N * K // 2 + N * (K // gs) * 2 * (1 + has_zero) + 2 * M * K + 2 * M * N
     if op == "w8a8":
@@ -109,6 +144,24 @@ def load_peaks():
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def roofline_of(op, M, K, N, hz, ms, peaks, burst=True):
+    """Which roof bounds the shape (arithmetic intensity against the ridge of the measured
+    peaks) and the achieved fraction of it for a call of `ms` milliseconds. int8 contractions
+    take the measured bf16 peak times the nominal dense int8 / bf16 ratio (2)."""
+    fl = shape_flops(M, K, N)
+    by = shape_bytes(op, M, K, N, hz)
+    tscale = 2.0 if op in ("w8a8", "w2a8") else 1.0
+    tpeak = tscale * (peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"])
+    ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if fl / by >= ridge:
+        ach = fl / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(tpeak, 1),
+                "unit": UNITS[op], "frac": round(ach / tpeak, 4)}
+    ach = by / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4)}
 
 
 class ClockSampler:
@@ -204,77 +257,252 @@ def barrier(world: int, device=None):
             dist.barrier()
 
 
+def tile_samples(M: int, N: int, seed: int, tm: int = 128, tn: int = 128):
+    """(m, n) positions of C to check: one seeded random element inside every tm x tn tile
+    (the ragged edge tiles included) plus the four corners of C."""
+    rng = np.random.default_rng(seed)
+    mt, nt = -(-M // tm), -(-N // tn)
+    i = np.repeat(np.arange(mt, dtype=np.int64), nt)
+    j = np.tile(np.arange(nt, dtype=np.int64), mt)
+    hm = np.minimum(tm, M - i * tm)
+    hn = np.minimum(tn, N - j * tn)
+    ms = i * tm + (rng.random(i.size) * hm).astype(np.int64)
+    ns = j * tn + (rng.random(j.size) * hn).astype(np.int64)
+    ms = np.concatenate([ms, np.array([0, 0, M - 1, M - 1], dtype=np.int64)])
+    ns = np.concatenate([ns, np.array([0, N - 1, 0, N - 1], dtype=np.int64)])
+    return ms, ns
+
+
+# ---- parity leg: the timed outputs against the host oracle --------------------------------------
+
+def parity_check(op, h, C, M, K, N, hz, seed):
+    """Compare sampled elements of the device result C (torch, [M, N]) with the host oracle on
+    the same seeded host inputs `h`. Returns {"checked", "bad", ...}."""
+    import torch
+    import oracle
+    ms, ns = tile_samples(M, N, seed)
+    idx = torch.from_numpy(ms * N + ns).to(C.device)
+    got = C.reshape(-1).index_select(0, idx).cpu().numpy()
+    if op == "w4a16":
+        if "Wq_oracle" not in h:
+            h["Wq_oracle"] = oracle.pack_int4(h["codes"])
+        ref = oracle.w4a16_at(h["A"], h["Wq_oracle"], h["scales"], h["zeros"], K, GS, ms, ns)
+    elif op == "dense":
+        ref = oracle.dense_f16_at(h["A"], h["W"], ms, ns)
+    elif op == "w8a8":
+        ref = oracle.w8a8_at(h["A"], h["W"], ms, ns)
+    else:
+        if "Wq_oracle" not in h:
+            h["Wq_oracle"] = oracle.pack_int2(h["Wv"])
+        ref = oracle.w2a8_at(h["A"], h["Wq_oracle"], ms, ns)
+    if op in ("w8a8", "w2a8"):
+        bad = int(np.count_nonzero(got.astype(np.int64) != ref))
+        return {"checked": int(ms.size), "bad": bad, "rule": "bit-exact"}
+    g = got.astype(np.float64)
+    err = np.abs(g - ref)
+    bad = int(np.count_nonzero(~(err <= oracle.ATOL + oracle.RTOL * np.abs(ref))))
+    nr = float(np.linalg.norm(ref))
+    frob = float(np.linalg.norm(g - ref)) / nr if nr > 0 else float(np.linalg.norm(g - ref))
+    if frob > oracle.FROB:
+        bad = max(bad, 1)
+    return {"checked": int(ms.size), "bad": bad, "frob": float(f"{frob:.3e}"),
+            "rule": "|d| <= 0.02 + 0.01|ref|, frob <= 5e-3"}
+
+
+def merge_parity(items):
+    out = {"checked": 0, "bad": 0}
+    for p in items:
+        if p is None:
+            continue
+        out["checked"] += p["checked"]
+        out["bad"] += p["bad"]
+    return out
+
+
 # ---- our arm ----------------------------------------------------------------------------------------
 
-def OP_CODES_table():
+def op_code(op):
     import gemv_w4a16_w8a8_b200 as qg
     return {"w4a16": qg.OP_W4A16, "w8a8": qg.OP_W8A8, "w2a8": qg.OP_W2A8,
-            "dense": qg.OP_DENSE_F16}
+            "dense": qg.OP_DENSE_F16}[op]
 
 
-OP_CODES = {k: (lambda k=k: OP_CODES_table()[k]) for k in ("w4a16", "w8a8", "w2a8", "dense")}
+def host_inputs(op, M, K, N, hz, seed):
+    from gemv_w4a16_w8a8_b200 import synth
+    if op == "w4a16":
+        return synth.w4a16_inputs(M, N, K, GS, bool(hz), seed=seed)
+    if op == "w8a8":
+        return synth.w8a8_inputs(M, N, K, seed=seed)
+    if op == "w2a8":
+        return synth.w2a8_inputs(M, N, K, seed=seed)
+    return synth.dense_inputs(M, N, K, seed=seed)
 
 
-def prepare_shape(op, M, K, N, hz, gs, seed, dev):
+def prepare_shape(op, M, K, N, hz, seed, dev, pinned=True):
     """Seeded inputs of one shape in HBM (weights replicated into enough copies, >= 3x L2 in
     total, that consecutive calls never find theirs in L2), plus page-locked host copies of A
-    and C for the end-to-end form."""
+    and C for the end-to-end form. The host arrays stay in sp["h"] for the parity leg."""
     import torch
     import gemv_w4a16_w8a8_b200 as qg
-    from gemv_w4a16_w8a8_b200 import synth
-    sp = {"M": M, "K": K, "N": N}
+    h = host_inputs(op, M, K, N, hz, seed)
+    sp = {"M": M, "K": K, "N": N, "hz": hz, "seed": seed, "h": h}
     if op == "w4a16":
-        d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=seed)
-        A_np = d["A"]
-        codes = torch.from_numpy(d["codes"]).to(dev)
+        codes = torch.from_numpy(h["codes"]).to(dev)
         W0 = qg.quant_pack_int4(codes)
         del codes
-        sp["S"] = torch.from_numpy(d["scales"]).to(dev)
-        sp["Z"] = torch.from_numpy(d["zeros"]).to(dev) if hz else None
+        sp["S"] = torch.from_numpy(h["scales"]).to(dev)
+        sp["Z"] = torch.from_numpy(h["zeros"]).to(dev) if hz else None
         c_dtype, wbytes = torch.float16, N * K // 2
     elif op == "w8a8":
-        d = synth.w8a8_inputs(M, N, K, seed=seed)
-        A_np = d["A"]
-        W0 = torch.from_numpy(d["W"]).to(dev)
+        W0 = torch.from_numpy(h["W"]).to(dev)
         c_dtype, wbytes = torch.int32, N * K
     elif op == "w2a8":
-        d = synth.w2a8_inputs(M, N, K, seed=seed)
-        A_np = d["A"]
-        W0 = qg.quant_pack_int2(torch.from_numpy(d["Wv"]).to(dev))
+        W0 = qg.quant_pack_int2(torch.from_numpy(h["Wv"]).to(dev))
         c_dtype, wbytes = torch.int32, N * K // 4
     else:
-        d = synth.dense_inputs(M, N, K, seed=seed)
-        A_np = d["A"]
-        W0 = torch.from_numpy(d["W"]).to(dev)
+        W0 = torch.from_numpy(h["W"]).to(dev)
         c_dtype, wbytes = torch.float16, 2 * N * K
     n_sets = max(1, min(64, math.ceil(3 * L2_BYTES / wbytes)))
-    sp.update({"A": torch.from_numpy(A_np).to(dev), "W": [W0] + [W0.clone() for _ in range(n_sets - 1)],
-               "C": torch.empty((M, N), dtype=c_dtype, device=dev), "n_sets": n_sets,
-               "A_host": torch.from_numpy(A_np).pin_memory(),
-               "C_host": torch.empty((M, N), dtype=c_dtype).pin_memory()})
+    sp.update({"A": torch.from_numpy(h["A"]).to(dev),
+               "W": [W0] + [W0.clone() for _ in range(n_sets - 1)],
+               "C": torch.empty((M, N), dtype=c_dtype, device=dev), "n_sets": n_sets})
+    if pinned:
+        sp["A_host"] = torch.from_numpy(h["A"]).pin_memory()
+        sp["C_host"] = torch.empty((M, N), dtype=c_dtype).pin_memory()
     return sp
 
 
-def matmul(op, sp, W, gs, A=None, C=None):
+def matmul(op, sp, W, split_k=0, A=None, C=None):
     """One call of the library's entry point for this op."""
     import gemv_w4a16_w8a8_b200 as qg
     A = sp["A"] if A is None else A
     C = sp["C"] if C is None else C
     if op == "w4a16":
-        qg.qgemm_w4a16(A, W, sp["S"], sp["Z"], C=C, group_size=gs)
+        qg.qgemm_w4a16(A, W, sp["S"], sp["Z"], C=C, group_size=GS, split_k=split_k)
     elif op == "w8a8":
-        qg.qgemm_w8a8(A, W, C=C)
+        qg.qgemm_w8a8(A, W, C=C, split_k=split_k)
     elif op == "w2a8":
-        qg.qgemm_w2a8(A, W, C=C)
+        qg.qgemm_w2a8(A, W, C=C, split_k=split_k)
     else:
-        qg.qgemm_dense_f16(A, W, C=C)
+        qg.qgemm_dense_f16(A, W, C=C, split_k=split_k)
+
+
+def tune_shape(op, sp, hz, no_tune, reps):
+    import gemv_w4a16_w8a8_b200 as qg
+    M, K, N = sp["M"], sp["K"], sp["N"]
+    g_op = GS if op == "w4a16" else -1
+    if no_tune:
+        return qg.qgemm_plan(op_code(op), M, N, K, g_op, hz)
+    return qg.qgemm_tune(op_code(op), sp["A"], sp["W"][0], sp.get("S"), sp.get("Z"), sp["C"],
+                         M, N, K, g_op, hz, reps=reps)
+
+
+def time_shape(op, sp, split_k=0, reps=None):
+    """Mean device time (ms) of one call from a CUDA graph of back-to-back calls, weight sets
+    cycling. The graph is replayed once untimed first."""
+    import torch
+    n = sp["n_sets"]
+    reps = reps or min(64, max(n, 20))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for r in range(reps):
+            matmul(op, sp, sp["W"][r % n], split_k)
+    g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / reps
+
+
+CFG_KEYS = ("path", "rows", "bm", "bn", "bk", "stages", "split_k", "swap_ab")
+
+
+def shape_row(op, sp, ms, cfg, peaks, parity, split_req="tuned"):
+    M, K, N, hz = sp["M"], sp["K"], sp["N"], sp["hz"]
+    by, fl = shape_bytes(op, M, K, N, hz), shape_flops(M, K, N)
+    roof = roofline_of(op, M, K, N, hz, ms, peaks)
+    return {"shape_mkn": [M, K, N], "has_zero": hz, "split_k_req": split_req,
+            "cfg": {k: cfg[k] for k in CFG_KEYS}, "us": round(ms * 1e3, 2),
+            "gbs": round(by / (ms * 1e-3) / 1e9, 1),
+            ("tops" if op in ("w8a8", "w2a8") else "tflops"): round(fl / (ms * 1e-3) / 1e12, 2),
+            "bound": roof["bound"], "frac": roof["frac"], "parity": parity}
+
+
+def run_extras(args, dev, peaks, headline_sps, deadline):
+    """The other benchmark configurations, shape by shape (see the module docstring)."""
+    import torch
+    import gemv_w4a16_w8a8_b200 as qg
+    out, sweep, skipped = {}, [], []
+    for name, wl_name, splits, do_sweep in EXTRAS:
+        if time.time() > deadline:
+            skipped.append(name)
+            continue
+        wl = WORKLOADS[wl_name]
+        op, hz = wl["op"], wl["has_zero"]
+        rows = []
+        for si, (M, K, N) in enumerate(wl["shapes"]):
+            sp = prepare_shape(op, M, K, N, hz, 7000 + 100 * si + hz, dev, pinned=False)
+            g_op = GS if op == "w4a16" else -1
+            for s in splits:   # the planner's path at the stated split, before the search
+                cfg = qg.qgemm_plan(op_code(op), M, N, K, g_op, hz, s)
+                ms = time_shape(op, sp, split_k=s)
+                par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"])
+                rows.append(shape_row(op, sp, ms, cfg, peaks, par, split_req=s))
+            cfg = tune_shape(op, sp, hz, args.no_tune, args.tune_reps)
+            ms = time_shape(op, sp)
+            par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"])
+            rows.append(shape_row(op, sp, ms, cfg, peaks, par))
+            if do_sweep:
+                sweep += stage_sweep(op, sp, cfg, peaks)
+            qg.qgemm_sync_check()
+            del sp
+            torch.cuda.empty_cache()
+        out[name] = {"op": op, "has_zero": hz, "per_shape": rows}
+    # the headline's own large-M W4A16 shapes (zero points) in the stage sweep
+    for sp in headline_sps:
+        if sp["M"] >= 512 and time.time() <= deadline:
+            sweep += stage_sweep("w4a16", sp, sp["cfg"], peaks)
+    return out, sweep, skipped
+
+
+def stage_sweep(op, sp, tuned, peaks):
+    """Pipeline depth 2..5 of the tensor-core kernel on this shape, the tuned tile and split
+    kept; each depth timed and parity-checked, then the tuned configuration restored."""
+    import gemv_w4a16_w8a8_b200 as qg
+    M, K, N, hz = sp["M"], sp["K"], sp["N"], sp["hz"]
+    g_op = GS if op == "w4a16" else -1
+    rows = []
+    if tuned["path"] != qg.PATH_TC:
+        return rows
+    for st in SWEEP_STAGES:
+        cfg = dict(tuned)
+        cfg["stages"] = st
+        try:
+            qg.qgemm_set_config(op_code(op), M, N, K, g_op, hz, cfg)
+        except qg.QGemmError:
+            rows.append({"op": op, "shape_mkn": [M, K, N], "has_zero": hz, "stages": st,
+                         "cfg": cfg, "us": None, "note": "does not fit shared memory"})
+            continue
+        ms = time_shape(op, sp, reps=max(4, min(20, sp["n_sets"])))
+        par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"] + st)
+        r = shape_row(op, sp, ms, cfg, peaks, par)
+        r.update({"op": op, "stages": st})
+        rows.append(r)
+    qg.qgemm_set_config(op_code(op), M, N, K, g_op, hz, tuned)
+    return rows
 
 
 def run_ours(args, world, rank, local):
     import torch
     import gemv_w4a16_w8a8_b200 as qg
-    from gemv_w4a16_w8a8_b200 import synth
 
+    t_start = time.time()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -283,35 +511,28 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     wl = WORKLOADS[args.workload]
-    op, hz, gs = wl["op"], wl["has_zero"], 128
+    op, hz = wl["op"], wl["has_zero"]
     shapes = wl["shapes"]
     peaks = load_peaks()
 
     # inputs: one A per shape; weights: each shape's packed matrix replicated into enough
     # copies (>= 3x L2 in total) that consecutive calls of a shape never find theirs in L2
-    per_shape = [prepare_shape(op, M, K, N, hz, gs, 1000 * si, dev)
+    per_shape = [prepare_shape(op, M, K, N, hz, 1000 * si, dev)
                  for si, (M, K, N) in enumerate(shapes)]
     torch.cuda.synchronize()
 
     # configuration search (once per shape, before timing)
     tuned = []
     for sp in per_shape:
-        M, K, N = sp["M"], sp["K"], sp["N"]
-        g_op = gs if op == "w4a16" else -1
-        if args.no_tune:
-            cfg = qg.qgemm_plan(OP_CODES[op](), M, N, K, g_op, hz)
-        else:
-            cfg = qg.qgemm_tune(OP_CODES[op](), sp["A"], sp["W"][0], sp.get("S"), sp.get("Z"),
-                                sp["C"], M, N, K, g_op, hz, reps=args.tune_reps)
+        cfg = tune_shape(op, sp, hz, args.no_tune, args.tune_reps)
         sp["cfg"] = cfg
-        tuned.append({"shape": [M, K, N], **{k: cfg[k] for k in ("path", "rows", "bm", "bn",
-                                                                   "bk", "stages", "split_k")}})
+        tuned.append({"shape": [sp["M"], sp["K"], sp["N"]], **{k: cfg[k] for k in CFG_KEYS}})
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
 
     def call(sp, i):
-        matmul(op, sp, sp["W"][i % sp["n_sets"]], gs)
+        matmul(op, sp, sp["W"][i % sp["n_sets"]])
 
     n_sets = max(sp["n_sets"] for sp in per_shape)
 
@@ -329,8 +550,7 @@ def run_ours(args, world, rank, local):
                 call(sp, w)
         graphs.append(g)
     # per-shape graphs (R back-to-back calls, weight sets cycling) for the per-call timings
-    reps = max(n_sets, 20)
-    reps = min(reps, 64)
+    reps = min(max(n_sets, 20), 64)
     shape_graphs = []
     for sp in per_shape:
         g = torch.cuda.CUDAGraph()
@@ -379,6 +599,18 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         shape_ms.append(e0.elapsed_time(e1) / reps)
     clk.__exit__(None, None, None)
+    del graphs, shape_graphs
+
+    # no kernel of the timed region may have given up a bounded wait
+    device_error = None
+    try:
+        qg.qgemm_sync_check()
+    except qg.QGemmError as e:
+        device_error = str(e)
+
+    # parity of what was timed: every shape's output under its tuned configuration
+    parity_rows = [parity_check(op, sp["h"], sp["C"], sp["M"], sp["K"], sp["N"], hz, sp["seed"])
+                   for sp in per_shape]
 
     flops_step = sum(shape_flops(s["M"], s["K"], s["N"]) for s in per_shape)
     bytes_step = sum(shape_bytes(op, s["M"], s["K"], s["N"], hz) for s in per_shape)
@@ -386,29 +618,14 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
 
     # ---- end to end: host A in, host C out, through the same entry point ----
-    e2e = run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step)
+    e2e = run_e2e(args, op, per_shape, hz, stream, world, dev, flops_step)
 
     # ---- roofline of the dominant call ----
     j = int(np.argmax(shape_ms))
     sp = per_shape[j]
     M, K, N = sp["M"], sp["K"], sp["N"]
-    fl = shape_flops(M, K, N)
-    by = shape_bytes(op, M, K, N, hz)
-    ms = shape_ms[j]
-    intensity = fl / by
     timed_alone = total_ms < 1000.0
-    # int8 contractions: the measured bf16 peak times the nominal dense int8 / bf16 ratio (2)
-    tscale = 2.0 if op in ("w8a8", "w2a8") else 1.0
-    tpeak = tscale * (peaks["bf16_tflops"] if timed_alone else peaks["bf16_tflops_sustained"])
-    ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)   # flop per byte
-    if intensity >= ridge:
-        achieved = fl / (ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(tpeak, 1),
-                "unit": UNITS[op], "frac": round(achieved / tpeak, 4)}
-    else:
-        achieved = by / (ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    roof = roofline_of(op, M, K, N, hz, shape_ms[j], peaks, burst=timed_alone)
     if args.traffic is not None:
         roof["traffic"] = args.traffic
     elif (M, K, N) in TRAFFIC_BYTES and sp["cfg"]["path"] == 2 and sp["cfg"]["bn"] == 256 and \
@@ -420,17 +637,34 @@ def run_ours(args, world, rank, local):
     roof["kernel_shape"] = [M, K, N]
     roof["peak_source"] = (f"{peaks['source']} "
                            f"({'burst' if timed_alone else 'sustained'} for tensor peaks"
-                           + (", x2 for int8 (nominal dense int8 / bf16)" if tscale != 1 else "")
-                           + ")")
+                           + (", x2 for int8 (nominal dense int8 / bf16)"
+                              if op in ("w8a8", "w2a8") else "") + ")")
 
-    details = []
-    for s, t in zip(per_shape, shape_ms):
-        fl_s = shape_flops(s["M"], s["K"], s["N"])
-        by_s = shape_bytes(op, s["M"], s["K"], s["N"], hz)
-        details.append({"shape_mkn": [s["M"], s["K"], s["N"]], "us": round(t * 1e3, 2),
-                        "gbs": round(by_s / (t * 1e-3) / 1e9, 1),
-                        "tflops": round(fl_s / (t * 1e-3) / 1e12, 2),
-                        "hbm_frac": round(by_s / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
+    details = [shape_row(op, s, t, s["cfg"], peaks, p)
+               for s, t, p in zip(per_shape, shape_ms, parity_rows)]
+
+    l2_sets = [s["n_sets"] for s in per_shape]
+    extras, sweep, skipped = {}, [], []
+    if not args.no_extras and world == 1:
+        deadline = time.time() + args.extras_budget
+        # the headline's device buffers stay for the stage sweep of its large shapes; the rest go
+        for s in per_shape:
+            s.pop("A_host", None)
+            s.pop("C_host", None)
+        big = [s for s in per_shape if s["M"] >= 512]
+        for s in per_shape:
+            if s["M"] < 512:
+                s.clear()
+        torch.cuda.empty_cache()
+        extras, sweep, skipped = run_extras(args, dev, peaks, big, deadline)
+        try:
+            qg.qgemm_sync_check()
+        except qg.QGemmError as e:
+            device_error = device_error or str(e)
+
+    parity = merge_parity(parity_rows + ([e2e.get("parity")] if e2e.get("parity") else []))
+    extra_parity = merge_parity([r["parity"] for c in extras.values() for r in c["per_shape"]] +
+                                [r.get("parity") for r in sweep])
 
     out = {
         "metric": METRICS[op],
@@ -438,7 +672,7 @@ def run_ours(args, world, rank, local):
         "unit": UNITS[op],
         "n_gpus": world,
         "steps": args.steps,
-        "warmup": warm_steps,
+        "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True,
         "scaling": "weak",
@@ -446,12 +680,13 @@ def run_ours(args, world, rank, local):
         "dtype": DTYPES[op],
         "data": "synthetic",
         "config": {"workload": args.workload, "op": op, "shapes_mkn": [list(s) for s in shapes],
-                   "group_size": gs, "has_zero": hz, "parallelism": f"replicas{world}",
+                   "group_size": GS, "has_zero": hz, "parallelism": f"replicas{world}",
                    "l2": "rotating weight copies per shape, >= 3x L2 between reuses "
-                         f"({[sp['n_sets'] for sp in per_shape]})",
+                         f"({l2_sets})",
                    "tuned": tuned},
         "hbm_gbs_effective": round(world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9, 1),
         "per_shape": details,
+        "parity": parity,
         "roofline": roof,
         "e2e": e2e,
         "clocks": clk.summary(),
@@ -460,15 +695,24 @@ def run_ours(args, world, rank, local):
                    "warmup_steps_run": warm_steps},
         "gpu_launches": args.steps * len(per_shape),
     }
+    if extras or sweep:
+        out["configs"] = extras
+        out["stage_sweep"] = sweep
+        out["configs_parity"] = extra_parity
+        if skipped:
+            out["configs_skipped"] = skipped
+    if device_error:
+        out["device_error"] = device_error
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_budget)
+    out["wall_s"] = round(time.time() - t_start, 1)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return out
 
 
-def run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step):
+def run_e2e(args, op, per_shape, hz, stream, world, dev, flops_step):
     """The same step end to end: A from page-locked host memory in, C to page-locked host
     memory out, every shape every step. W4A16 goes through the host-buffer entry point, which
     streams chunks of tokens through a device workspace so that both copy directions overlap
@@ -488,10 +732,10 @@ def run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step):
             W = sp["W"][i % len(sp["W"])]
             if op == "w4a16":
                 qg.qgemm_w4a16_host(sp["A_host"], W, sp["S"], sp["Z"], sp["C_host"], ws,
-                                    group_size=gs)
+                                    group_size=GS)
             else:
                 sp["A"].copy_(sp["A_host"], non_blocking=True)
-                matmul(op, sp, W, gs)
+                matmul(op, sp, W)
                 sp["C_host"].copy_(sp["C"], non_blocking=True)
 
     one(0)
@@ -506,12 +750,15 @@ def run_e2e(args, op, per_shape, gs, hz, stream, world, dev, flops_step):
     e1.record(stream)
     torch.cuda.synchronize()
     value, ms = job_throughput(e0.elapsed_time(e1), flops_step, steps, world, dev)
+    # the host-side results of the last step, sampled against the oracle
+    par = merge_parity([parity_check(op, sp["h"], sp["C_host"], sp["M"], sp["K"], sp["N"], hz,
+                                     sp["seed"] + 1) for sp in per_shape])
     path = ("qgemm_w4a16_host (pinned host A and C, chunks of up to 2048 tokens, copies in both "
             "directions overlapped with the matmul)" if op == "w4a16" else
             "pinned host A copied in, the call, C copied out, on one stream")
     return {"value": round(value, 3), "unit": UNITS[op],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": round(ms / steps, 3), "path": path}
+            "ms_per_step": round(ms / steps, 3), "path": path, "parity": par}
 
 
 # ---- oracle arm ------------------------------------------------------------------------------------
@@ -527,7 +774,7 @@ def oracle_sample_rates(workload: str, budget_s: float, seed: int = 0):
     import oracle
     from gemv_w4a16_w8a8_b200 import synth
     wl = WORKLOADS[workload]
-    hz, gs = wl["has_zero"], 128
+    hz = wl["has_zero"]
     threads = oracle.max_threads()
     per = budget_s / len(wl["shapes"])
     out = []
@@ -538,7 +785,7 @@ def oracle_sample_rates(workload: str, budget_s: float, seed: int = 0):
         key = (op, m_s, n_all, K, hz, seed + si)
         if key not in _ORACLE_INPUTS:
             if op == "w4a16":
-                d = synth.w4a16_inputs(m_s, n_all, K, gs, bool(hz), seed=seed + si)
+                d = synth.w4a16_inputs(m_s, n_all, K, GS, bool(hz), seed=seed + si)
                 d["Wq"] = oracle.pack_int4(d["codes"])
             elif op == "w8a8":
                 d = synth.w8a8_inputs(m_s, n_all, K, seed=seed + si)
@@ -553,7 +800,7 @@ def oracle_sample_rates(workload: str, budget_s: float, seed: int = 0):
         def run_slice(n):
             if op == "w4a16":
                 oracle.w4a16(d["A"], d["Wq"][:n], d["scales"][:n],
-                             None if d["zeros"] is None else d["zeros"][:n], K, gs, nthreads=threads)
+                             None if d["zeros"] is None else d["zeros"][:n], K, GS, nthreads=threads)
             elif op == "w8a8":
                 oracle.w8a8(d["A"], d["W"][:n], nthreads=threads)
             elif op == "w2a8":
@@ -583,7 +830,8 @@ def cpu_baseline(workload: str, budget_s: float = 15.0):
     return {"value": total / est_s / 1e12, "unit": UNITS[wl["op"]], "cores": threads, "kind": "oracle",
             "sample": "; ".join(desc for _, _, desc in rates) +
                       f" (fp64 oracle, {sum(t for _, t, _ in rates):.1f} s wall on {threads} threads; "
-                      f"each shape's rate applied to its full FLOPs)"}
+                      f"each shape's rate applied to its full FLOPs)",
+            "extrapolated": True}
 
 
 def run_reference(args, world, rank):
@@ -595,12 +843,14 @@ def run_reference(args, world, rank):
     for _ in range(max(0, args.warmup)):
         oracle_sample_rates(args.workload, per_step_budget / 4)
     est = []
+    sampled = []
     threads = 1
     samples = ""
     for _ in range(args.steps):
         rates, threads = oracle_sample_rates(args.workload, per_step_budget)
         est.append(sum(shape_flops(M, K, N) / (f / t)
                        for (M, K, N), (f, t, _) in zip(wl["shapes"], rates)))
+        sampled.append(sum(t for _, t, _ in rates))
         samples = "; ".join(d for _, _, d in rates)
     ms_per_step = 1e3 * statistics.mean(est)
     value = total_flops / (ms_per_step * 1e-3) / 1e12
@@ -609,13 +859,17 @@ def run_reference(args, world, rank):
         "metric": METRICS[wl["op"]],
         "value": value, "unit": UNITS[wl["op"]], "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "extrapolated": True,
+        "sample_s_per_step": round(statistics.mean(sampled), 3),
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "op": wl["op"],
-                   "shapes_mkn": [list(s) for s in wl["shapes"]], "group_size": 128,
+                   "shapes_mkn": [list(s) for s in wl["shapes"]], "group_size": GS,
                    "has_zero": wl["has_zero"], "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": UNITS[wl["op"]], "cores": threads, "kind": "oracle",
                          "sample": samples + " per step; each shape's sampled rate applied to "
-                                             "its full FLOPs"},
+                                             "its full FLOPs (ms_per_step is that extrapolation; "
+                                             "sample_s_per_step is the measured wall time)",
+                         "extrapolated": True},
         "e2e": {"value": value, "unit": UNITS[wl["op"]], "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -632,6 +886,10 @@ def main(argv=None):
     ap.add_argument("--tune-reps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time only the headline workload")
+    ap.add_argument("--extras-budget", type=float, default=240.0,
+                    help="seconds after which the remaining extra configurations are skipped")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args(argv)
@@ -642,6 +900,11 @@ def main(argv=None):
         out = run_ours(args, world, rank, local)
     if rank == 0 and out is not None:
         print(json.dumps(out), flush=True)
+    if out is not None and out.get("impl") != "reference":
+        failed = (out.get("device_error") or out["parity"]["bad"] or
+                  out.get("configs_parity", {}).get("bad", 0))
+        if failed:
+            return 3
     return 0
 
 

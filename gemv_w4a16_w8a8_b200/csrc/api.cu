@@ -463,9 +463,9 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
         const int rows_w2[] = {1, 2, 4, 8, 16, 32, 64};
         const int *rows = p.op == QG_OP_W4A16 ? rows16 : (p.op == QG_OP_W2A8 ? rows_w2 : rows_int);
         const int nrows = p.op == QG_OP_W4A16 ? 3 : (p.op == QG_OP_W2A8 ? 7 : 4);
-        const int stage_opts[5] = {0, 2, 3, 4, 6};     // 0: register-prefetch kernel
+        const int stage_opts[6] = {0, 2, 3, 4, 5, 6};  // 0: register-prefetch kernel
         for (int r = 0; r < nrows; ++r)
-            for (int st = 0; st < (p.op == QG_OP_W8A8 ? 1 : 5); ++st)
+            for (int st = 0; st < (p.op == QG_OP_W8A8 ? 1 : 6); ++st)
                 for (int s = 1; s <= 16; s *= 2) {
                     c.rows = rows[r];
                     c.stages = stage_opts[st];
@@ -475,7 +475,7 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
         if (p.op == QG_OP_W4A16 && p.M == 1) {
             // one token on the FMA pipe (TMA-fed kernel, bn = 1)
             for (int rows : {32, 64, 128})
-                for (int st : {2, 3, 4, 6})
+                for (int st : {2, 3, 4, 5, 6})
                     for (int s = 1; s <= 16; s *= 2) {
                         c.rows = rows;
                         c.bn = 1;
@@ -1013,30 +1013,65 @@ qg_status qgemm_tune(int op, const void *A, const void *W, const void *scales,
         cudaGetLastError();
         return QG_ERR_CUDA;
     }
+    // A timeout raised by work queued before the search belongs to that work's caller: report
+    // it now instead of charging it to a candidate (or losing it when the word is cleared).
+    unsigned int word = 0;
+    const unsigned int zero = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&word, g_qgemm_error_word, sizeof(word)) != cudaSuccess) {
+        cudaGetLastError();
+        cudaEventDestroy(e0);
+        cudaEventDestroy(e1);
+        return QG_ERR_CUDA;
+    }
+    if (word) {
+        cudaEventDestroy(e0);
+        cudaEventDestroy(e1);
+        return QG_ERR_DEVICE_TIMEOUT;
+    }
     float best_ms = 1e30f;
+    bool have_winner = false;
     qgemm_config_t winner = cands[0];
     qg_status result = QG_OK;
     for (const qgemm_config_t &c : cands) {
         for (int i = 0; i < 2 && result == QG_OK; ++i) result = run(p, c, d, stream);
         if (result != QG_OK) break;
-        cudaEventRecord(e0, stream);
+        if (cudaEventRecord(e0, stream) != cudaSuccess) result = QG_ERR_CUDA;
         for (int i = 0; i < reps && result == QG_OK; ++i) result = run(p, c, d, stream);
-        cudaEventRecord(e1, stream);
+        if (result == QG_OK && cudaEventRecord(e1, stream) != cudaSuccess) result = QG_ERR_CUDA;
         if (result != QG_OK || cudaEventSynchronize(e1) != cudaSuccess) {
             if (result == QG_OK) result = QG_ERR_CUDA;
             break;
         }
         float ms = 0.f;
-        cudaEventElapsedTime(&ms, e0, e1);
+        if (cudaEventElapsedTime(&ms, e0, e1) != cudaSuccess) {
+            result = QG_ERR_CUDA;
+            break;
+        }
+        // a candidate whose kernels gave up a bounded wait is dropped, and the word cleared so
+        // that the next candidate (and later callers) start clean
+        if (cudaMemcpyFromSymbol(&word, g_qgemm_error_word, sizeof(word)) != cudaSuccess) {
+            result = QG_ERR_CUDA;
+            break;
+        }
+        if (word) {
+            if (cudaMemcpyToSymbol(g_qgemm_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+                result = QG_ERR_CUDA;
+                break;
+            }
+            continue;
+        }
         if (ms < best_ms) {
             best_ms = ms;
             winner = c;
+            have_winner = true;
         }
     }
     cudaEventDestroy(e0);
     cudaEventDestroy(e1);
     cudaGetLastError();
     if (result != QG_OK) return result;
+    if (!have_winner) return QG_ERR_DEVICE_TIMEOUT;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         ensure_cache_loaded_locked();

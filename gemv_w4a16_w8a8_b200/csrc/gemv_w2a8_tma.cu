@@ -243,6 +243,7 @@ cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned in
     case 2: return launch_one<RB, NT, 2>(p, c.split_k, err, stream);
     case 3: return launch_one<RB, NT, 3>(p, c.split_k, err, stream);
     case 4: return launch_one<RB, NT, 4>(p, c.split_k, err, stream);
+    case 5: return launch_one<RB, NT, 5>(p, c.split_k, err, stream);
     default: return launch_one<RB, NT, 6>(p, c.split_k, err, stream);
     }
 }
@@ -261,7 +262,7 @@ cudaError_t launch_rb(const Problem &p, const qgemm_config_t &c, unsigned int *e
 bool gemv_w2a8_tma_supports(const Problem &p, const qgemm_config_t &c)
 {
     return p.op == QG_OP_W2A8 && p.K % kKB == 0 && (c.rows == 16 || c.rows == 32 || c.rows == 64) &&
-           (c.stages == 2 || c.stages == 3 || c.stages == 4 || c.stages == 6) && c.split_k >= 1 &&
+           (c.stages >= 2 && c.stages <= 6) && c.split_k >= 1 &&
            c.split_k <= 64;
 }
 

@@ -451,6 +451,7 @@ cudaError_t launch_simt_stages(const Problem &p, const qgemm_config_t &c, unsign
     case 2: return launch_one<RB, 1, 2, true>(p, c.split_k, err, stream, wp, wc);
     case 3: return launch_one<RB, 1, 3, true>(p, c.split_k, err, stream, wp, wc);
     case 4: return launch_one<RB, 1, 4, true>(p, c.split_k, err, stream, wp, wc);
+    case 5: return launch_one<RB, 1, 5, true>(p, c.split_k, err, stream, wp, wc);
     default: return launch_one<RB, 1, 6, true>(p, c.split_k, err, stream, wp, wc);
     }
 }
@@ -463,6 +464,7 @@ cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned in
     case 2: return launch_one<RB, NT, 2>(p, c.split_k, err, stream, wp, wc);
     case 3: return launch_one<RB, NT, 3>(p, c.split_k, err, stream, wp, wc);
     case 4: return launch_one<RB, NT, 4>(p, c.split_k, err, stream, wp, wc);
+    case 5: return launch_one<RB, NT, 5>(p, c.split_k, err, stream, wp, wc);
     default: return launch_one<RB, NT, 6>(p, c.split_k, err, stream, wp, wc);
     }
 }
@@ -480,7 +482,7 @@ cudaError_t launch_rb(const Problem &p, const qgemm_config_t &c, unsigned int *e
 
 bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &c)
 {
-    const bool stages_ok = c.stages == 2 || c.stages == 3 || c.stages == 4 || c.stages == 6;
+    const bool stages_ok = (c.stages >= 2 && c.stages <= 6);
     const bool base = p.gs % kKB == 0 && p.K % kKB == 0 && stages_ok && c.split_k >= 1 &&
                       c.split_k <= 64;
     if (c.bn == 1)   // one token on the FMA pipe

@@ -15,12 +15,19 @@ def to_dev(a: np.ndarray) -> torch.Tensor:
 
 
 def sample_pairs(M, N, count, seed, K=None):
-    """(m, n) positions: every tile corner and edge plus seeded random ones."""
+    """(m, n) positions: every tile corner and edge, one seeded random element inside every
+    128 x 128 tile of C (so that a fault confined to some output tiles or persistent units is
+    seen), plus `count` seeded random ones."""
     rng = np.random.default_rng(seed)
     ms = [0, M - 1, M // 2, min(M - 1, 15), min(M - 1, 16), min(M - 1, 127), min(M - 1, 128)]
     ns = [0, N - 1, N // 2, min(N - 1, 127), min(N - 1, 128), min(N - 1, 255), min(N - 1, 256)]
     pm = [m for m in ms for _ in ns]
     pn = [n for _ in ms for n in ns]
+    mt, nt = -(-M // 128), -(-N // 128)
+    ti = np.repeat(np.arange(mt, dtype=np.int64), nt)
+    tj = np.tile(np.arange(nt, dtype=np.int64), mt)
+    pm += list(ti * 128 + (rng.random(ti.size) * np.minimum(128, M - ti * 128)).astype(np.int64))
+    pn += list(tj * 128 + (rng.random(tj.size) * np.minimum(128, N - tj * 128)).astype(np.int64))
     pm += list(rng.integers(0, M, count))
     pn += list(rng.integers(0, N, count))
     return np.array(pm, dtype=np.int64), np.array(pn, dtype=np.int64)

@@ -97,3 +97,36 @@ def test_every_workload_is_consistent():
         for M, K, N in wl["shapes"]:
             assert bench.shape_bytes(wl["op"], M, K, N, wl["has_zero"]) > 0
             assert bench.shape_flops(M, K, N) == 2.0 * M * N * K
+
+
+def test_tile_samples_cover_every_tile_in_bounds():
+    for M, N in [(1, 1), (1, 16384), (32, 300), (129, 257), (16384, 4096)]:
+        ms, ns = bench.tile_samples(M, N, seed=3)
+        assert ms.min() >= 0 and ns.min() >= 0 and ms.max() < M and ns.max() < N
+        tiles = set(zip((ms // 128).tolist(), (ns // 128).tolist()))
+        assert tiles == {(i, j) for i in range(-(-M // 128)) for j in range(-(-N // 128))}
+        for corner in [(0, 0), (0, N - 1), (M - 1, 0), (M - 1, N - 1)]:
+            assert corner in set(zip(ms.tolist(), ns.tolist()))
+
+
+def test_parity_leg_accepts_the_oracle_and_catches_a_planted_error():
+    """The bench's parity leg on CPU: the oracle's own result rounded to fp16 passes; the same
+    result with one element pushed past the tolerance, or an integer result off by one, fails."""
+    import numpy as np
+    import torch
+    import oracle
+    from gemv_w4a16_w8a8_b200 import synth
+    M, K, N = 3, 256, 200
+    h = synth.w4a16_inputs(M, N, K, 128, True, seed=5)
+    ref = oracle.w4a16(h["A"], oracle.pack_int4(h["codes"]), h["scales"], h["zeros"], K, 128)
+    C = torch.from_numpy(ref.astype(np.float16))
+    p = bench.parity_check("w4a16", dict(h), C, M, K, N, 1, seed=9)
+    assert p["bad"] == 0 and p["checked"] == 2 * 1 + 4
+    C2 = C.clone()
+    C2[M - 1, N - 1] += 0.5 + 0.02 * abs(float(C2[M - 1, N - 1]))
+    assert bench.parity_check("w4a16", dict(h), C2, M, K, N, 1, seed=9)["bad"] >= 1
+    e = synth.w8a8_inputs(2, 130, 64, seed=1)
+    Ci = torch.from_numpy(oracle.w8a8(e["A"], e["W"]).astype(np.int32))
+    assert bench.parity_check("w8a8", e, Ci, 2, 64, 130, 0, seed=2)["bad"] == 0
+    Ci[0, 0] += 1
+    assert bench.parity_check("w8a8", e, Ci, 2, 64, 130, 0, seed=2)["bad"] == 1
