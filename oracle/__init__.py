@@ -39,7 +39,8 @@ class Oracle:
         L.orc_half_to_double.restype = ctypes.c_double
         L.orc_half_to_double.argtypes = [ctypes.c_uint16]
         for name in ("orc_pack_int4", "orc_unpack_int4", "orc_pack_int2", "orc_unpack_int2",
-                     "orc_pack_int4_interleaved", "orc_unpack_int4_interleaved"):
+                     "orc_pack_int4_interleaved", "orc_unpack_int4_interleaved",
+                     "orc_pack_int2_interleaved", "orc_unpack_int2_interleaved"):
             getattr(L, name).argtypes = [_ptr, _ptr, _i64, _i64]
             getattr(L, name).restype = ctypes.c_int
         L.orc_decode_half.argtypes = [_ptr, _ptr, _i64]
@@ -154,6 +155,21 @@ class Oracle:
         N = packed.shape[0]
         out = np.empty((N, K), dtype=np.int8)
         _check(self.L.orc_unpack_int2(_p(packed), _p(out), N, K), "unpack_int2")
+        return out
+
+    def pack_int2_interleaved(self, vals: np.ndarray) -> np.ndarray:
+        vals = np.ascontiguousarray(vals, dtype=np.int8)
+        N, K = vals.shape
+        out = np.empty((N, K // 16), dtype=np.uint32)
+        _check(self.L.orc_pack_int2_interleaved(_p(vals), _p(out), N, K), "pack_int2_interleaved")
+        return out
+
+    def unpack_int2_interleaved(self, packed: np.ndarray, K: int) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        N = packed.shape[0]
+        out = np.empty((N, K), dtype=np.int8)
+        _check(self.L.orc_unpack_int2_interleaved(_p(packed), _p(out), N, K),
+               "unpack_int2_interleaved")
         return out
 
     # ---- matmuls ----------------------------------------------------------------------------
@@ -282,6 +298,8 @@ def pack_int4_interleaved(c): return get().pack_int4_interleaved(c)
 def unpack_int4_interleaved(p, K): return get().unpack_int4_interleaved(p, K)
 def pack_int2(v): return get().pack_int2(v)
 def unpack_int2(p, K): return get().unpack_int2(p, K)
+def pack_int2_interleaved(v): return get().pack_int2_interleaved(v)
+def unpack_int2_interleaved(p, K): return get().unpack_int2_interleaved(p, K)
 def w4a16(*a, **k): return get().w4a16(*a, **k)
 def w4a16_at(*a, **k): return get().w4a16_at(*a, **k)
 def dense_f16(*a, **k): return get().dense_f16(*a, **k)

@@ -135,6 +135,37 @@ int orc_pack_int2(const int8_t *vals, uint32_t *packed, int64_t N, int64_t K)
     return ORC_OK;
 }
 
+/*
+ * Interleaved int2 packing (the pre-shuffled layout): inside each word, value k = 16j + i sits in
+ * 2-bit field ILV2_POS[i] = 8 * (i / 8) + 2 * (i % 4) + (i % 8) / 4, i.e. fields 0..15 hold values
+ * 0, 4, 1, 5, 2, 6, 3, 7, 8, 12, 9, 13, 10, 14, 11, 15 of the word.
+ */
+static const int ILV2_POS[16] = {0, 2, 4, 6, 1, 3, 5, 7, 8, 10, 12, 14, 9, 11, 13, 15};
+
+int orc_pack_int2_interleaved(const int8_t *vals, uint32_t *packed, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 16) return ORC_BAD_ARGS;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 16; ++j) {
+            uint32_t word = 0;
+            for (int i = 0; i < 16; ++i)
+                word |= (uint32_t)((uint8_t)vals[n * K + 16 * j + i] & 3u) << (2 * ILV2_POS[i]);
+            packed[n * (K / 16) + j] = word;
+        }
+    return ORC_OK;
+}
+
+int orc_unpack_int2_interleaved(const uint32_t *packed, int8_t *vals, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 16) return ORC_BAD_ARGS;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            const int u = (int)((packed[n * (K / 16) + k / 16] >> (2 * ILV2_POS[k % 16])) & 3u);
+            vals[n * K + k] = (int8_t)(u - 4 * (u >> 1));
+        }
+    return ORC_OK;
+}
+
 /* field u in 0..3 read as a two's-complement 2-bit integer: u - 4 * (u >> 1) */
 static int int2_value(const uint32_t *packed, int64_t K, int64_t n, int64_t k)
 {

@@ -86,6 +86,26 @@ def test_pack_interleaved():
     check_pack_interleaved(oracle.get())
 
 
+def check_pack_int2_interleaved(orc):
+    for vals, word in _fixture_rows("pack_int2_interleaved.txt"):
+        got = orc.pack_int2_interleaved(np.array([vals], dtype=np.int8))
+        assert int(got[0, 0]) == word, (vals, hex(int(got[0, 0])))
+        back = orc.unpack_int2_interleaved(np.array([[word]], dtype=np.uint32), 16)
+        assert back.tolist() == [vals]
+    # the same values in both layouts: a fixed permutation of the 2-bit fields of every word
+    vals = synth.uniform_int((5, 128), -2, 1, 9, synth.TID_W, np.int8)
+    nat = orc.pack_int2(vals)
+    ilv = orc.pack_int2_interleaved(vals)
+    assert np.array_equal(orc.unpack_int2_interleaved(ilv, 128), vals)
+    perm = [0, 4, 1, 5, 2, 6, 3, 7, 8, 12, 9, 13, 10, 14, 11, 15]   # field f holds value perm[f]
+    for f, e in enumerate(perm):
+        assert np.array_equal((ilv >> (2 * f)) & 3, (nat >> (2 * e)) & 3)
+
+
+def test_pack_int2_interleaved():
+    check_pack_int2_interleaved(oracle.get())
+
+
 def test_pack_roundtrip_random():
     codes = synth.uniform_int((37, 256), 0, 15, 3, synth.TID_W, np.uint8)
     assert np.array_equal(oracle.unpack_int4(oracle.pack_int4(codes), 256), codes)
@@ -490,6 +510,13 @@ MUTANTS = [
     ("interleaved layout wrong", "static const int ILV_POS[8] = {0, 4, 1, 5, 2, 6, 3, 7};",
      "static const int ILV_POS[8] = {0, 1, 2, 3, 4, 5, 6, 7};"),
     ("interleaved unpack shift", "(4 * ILV_POS[k % 8])) & 0xF)", "(4 * (k % 8))) & 0xF)"),
+    ("int2 interleaved layout wrong",
+     "static const int ILV2_POS[16] = {0, 2, 4, 6, 1, 3, 5, 7, 8, 10, 12, 14, 9, 11, 13, 15};",
+     "static const int ILV2_POS[16] = {0, 4, 8, 12, 1, 5, 9, 13, 2, 6, 10, 14, 3, 7, 11, 15};"),
+    ("int2 interleaved unpack ignores the layout", "(2 * ILV2_POS[k % 16])) & 3u)",
+     "(2 * (k % 16))) & 3u)"),
+    ("int2 interleaved unpack sign", "vals[n * K + k] = (int8_t)(u - 4 * (u >> 1));",
+     "vals[n * K + k] = (int8_t)u;"),
     ("int2 pack not masked", "((uint8_t)vals[n * K + 16 * j + i] & 3u)",
      "((uint8_t)vals[n * K + 16 * j + i])"),
     ("half encoding ties away from zero", "(rem == halfway && (q & 1u))", "(rem == halfway)"),
@@ -506,7 +533,8 @@ MUTANTS = [
     ("requant multiplier by row", "* mult[n];", "* mult[m];"),
 ]
 
-PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
+PINS = [check_half_decoder, check_pack_fixtures, check_pack_interleaved,
+        check_pack_int2_interleaved, check_pack_masks_high_bits, check_w4_unit_scale_is_plain_matmul,
         check_w4_one_hot_reads_single_weight, check_w4_constant_closed_form,
         check_w4_per_channel_equals_one_group, check_w4_parallel_k_additivity,
         check_w4_elementwise_matches_full, check_dense_is_numpy_matmul,
