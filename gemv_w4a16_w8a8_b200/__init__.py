@@ -31,15 +31,16 @@ QG_ERR_SCRATCH_TOO_SMALL = 8
 QGEMM_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 OP_W4A16, OP_W8A8, OP_W2A8, OP_DENSE_F16, OP_W4A16_INTERLEAVED = 0, 1, 2, 3, 4
+OP_W2A8_INTERLEAVED = 5
 PATH_AUTO, PATH_GEMV, PATH_TC, PATH_STREAM = 0, 1, 2, 3
 
 # every symbol include/qgemm.h declares
 EXPORTS = (
     "qgemm_w4a16", "qgemm_w4a16_interleaved", "quant_pack_int4_interleaved", "qgemm_w4a16_splitk_f32", "qgemm_w4a16_workspace_bytes",
     "qgemm_w4a16_splitk_f32_noalloc", "qgemm_w4a16_host", "qgemm_w4a16_host_workspace_bytes",
-    "qgemm_w8a8", "qgemm_w2a8", "qgemm_dense_f16", "quant_pack_int4",
+    "qgemm_w8a8", "qgemm_w2a8", "qgemm_w2a8_interleaved", "qgemm_dense_f16", "quant_pack_int4",
     "quant_rtn_int4", "qgemm_w8a8_requant",
-    "quant_pack_int2", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
+    "quant_pack_int2", "quant_pack_int2_interleaved", "qgemm_plan", "qgemm_set_config", "qgemm_tune", "qgemm_save_configs",
     "qgemm_load_configs", "qgemm_clear_configs", "qgemm_sync_check", "qgemm_selftest_bounded_wait",
     "qgemm_status_string",
     "qgemm_version",
@@ -91,9 +92,11 @@ def lib() -> ctypes.CDLL:
         L.qgemm_w4a16_host_workspace_bytes.restype = ctypes.c_size_t
         L.qgemm_w8a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_w2a8.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.qgemm_w2a8_interleaved.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_dense_f16.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
         L.quant_pack_int4.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.quant_pack_int2.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
+        L.quant_pack_int2_interleaved.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, vp]
         L.qgemm_plan.argtypes = [i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(Config)]
         L.qgemm_set_config.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(Config)]
         L.qgemm_tune.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp,
@@ -330,6 +333,23 @@ def qgemm_w2a8(A, Wq, C=None, split_k: int = 0, stream=None):
     return C
 
 
+def qgemm_w2a8_interleaved(A, Wq, C=None, split_k: int = 0, stream=None):
+    """As qgemm_w2a8, with Wq from quant_pack_int2_interleaved."""
+    torch = _torch()
+    _need(A, torch.int8, 2, "A")
+    _need(Wq, (torch.int32, torch.uint32), 2, "Wq")
+    M, K = A.shape
+    N = Wq.shape[0]
+    if Wq.shape[1] * 16 != K:
+        raise ValueError("Wq must be [N, K/16]")
+    if C is None:
+        C = torch.empty((M, N), dtype=torch.int32, device=A.device)
+    _need(C, torch.int32, 2, "C")
+    _check(lib().qgemm_w2a8_interleaved(_ptr(A), _ptr(Wq), _ptr(C), M, N, K, -1, split_k, 0,
+                                        _stream(stream)), "qgemm_w2a8_interleaved")
+    return C
+
+
 def qgemm_dense_f16(A, W, C=None, split_k: int = 0, stream=None):
     """A fp16 [M,K]; W fp16 [N,K]. Returns C fp16 [M,N]."""
     torch = _torch()
@@ -383,6 +403,19 @@ def quant_pack_int2(vals, out=None, stream=None):
         out = torch.empty((N, K // 16), dtype=torch.int32, device=vals.device)
     _check(lib().quant_pack_int2(_ptr(vals), _ptr(out), 0, N, K, -1, 1, 0, _stream(stream)),
            "quant_pack_int2")
+    return out
+
+
+def quant_pack_int2_interleaved(vals, out=None, stream=None):
+    """vals int8 [N,K] (-2..1) -> int32 [N,K/16] in the interleaved layout (2-bit fields 0..15
+    of each word hold values 0,4,1,5,2,6,3,7, 8,12,9,13,10,14,11,15 of its sixteen)."""
+    torch = _torch()
+    _need(vals, torch.int8, 2, "vals")
+    N, K = vals.shape
+    if out is None:
+        out = torch.empty((N, K // 16), dtype=torch.int32, device=vals.device)
+    _check(lib().quant_pack_int2_interleaved(_ptr(vals), _ptr(out), 0, N, K, -1, 1, 0,
+                                             _stream(stream)), "quant_pack_int2_interleaved")
     return out
 
 

@@ -93,7 +93,7 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // Shape / flag rules shared by the matmul entry points, the planner and the tuner.
 qg_status check_shape(int op, int M, int N, int K, int group_size, int has_zero, int split_k)
 {
-    if (op < QG_OP_W4A16 || op > QG_OP_W4A16_INTERLEAVED) return QG_ERR_INVALID_ARG;
+    if (op < QG_OP_W4A16 || op > QG_OP_W2A8_INTERLEAVED) return QG_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
     if (split_k > kMaxSplit) return QG_ERR_INVALID_ARG;
     if (has_zero != 0 && has_zero != 1) return QG_ERR_INVALID_ARG;
@@ -108,9 +108,10 @@ qg_status check_shape(int op, int M, int N, int K, int group_size, int has_zero,
     }
     case QG_OP_W8A8:
     case QG_OP_W2A8:
+    case QG_OP_W2A8_INTERLEAVED:
         if (group_size != -1 && group_size != 0) return QG_ERR_INVALID_ARG;
         if (has_zero) return QG_ERR_INVALID_ARG;
-        if (K % (op == QG_OP_W2A8 ? 64 : 16)) return QG_ERR_UNSUPPORTED_SHAPE;
+        if (K % (op == QG_OP_W8A8 ? 16 : 64)) return QG_ERR_UNSUPPORTED_SHAPE;
         break;
     case QG_OP_DENSE_F16:
         if (has_zero) return QG_ERR_INVALID_ARG;
@@ -125,8 +126,9 @@ Problem make_problem(int op, const void *A, const void *W, const void *scales,
                      int has_zero)
 {
     Problem p;
-    p.op = op == QG_OP_W4A16_INTERLEAVED ? QG_OP_W4A16 : op;
-    p.interleaved = op == QG_OP_W4A16_INTERLEAVED ? 1 : 0;
+    p.op = op == QG_OP_W4A16_INTERLEAVED ? QG_OP_W4A16
+                                         : (op == QG_OP_W2A8_INTERLEAVED ? QG_OP_W2A8 : op);
+    p.interleaved = (op == QG_OP_W4A16_INTERLEAVED || op == QG_OP_W2A8_INTERLEAVED) ? 1 : 0;
     p.A = A;
     p.W = W;
     p.scales = scales;
@@ -150,8 +152,10 @@ bool supports(const Problem &p, const qgemm_config_t &c)
 {
     switch (c.path) {
     case QG_PATH_GEMV:
-        if (p.op == QG_OP_W4A16)
+        if (p.op == QG_OP_W4A16) {
+            if (c.bn == 2) return gemv_w4a16_h2_supports(p, c);
             return c.stages ? gemv_w4a16_tma_supports(p, c) : gemv_w4a16_supports(p, c);
+        }
         if (p.op == QG_OP_W2A8 && c.stages) return gemv_w2a8_tma_supports(p, c);
         if (p.op == QG_OP_W8A8 || p.op == QG_OP_W2A8) return gemv_int_supports(p, c);
         return false;
@@ -371,8 +375,10 @@ void ensure_cache_loaded_locked()
 
 Key key_of(const Problem &p)
 {
-    return Key(p.interleaved ? (int)QG_OP_W4A16_INTERLEAVED : p.op, p.M, p.N, p.K, p.gs,
-               p.has_zero);
+    const int op = !p.interleaved ? p.op
+                                  : (p.op == QG_OP_W2A8 ? (int)QG_OP_W2A8_INTERLEAVED
+                                                        : (int)QG_OP_W4A16_INTERLEAVED);
+    return Key(op, p.M, p.N, p.K, p.gs, p.has_zero);
 }
 
 qgemm_config_t choose(const Problem &p, int split_k, int sms)
@@ -410,7 +416,9 @@ qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStre
     }
     cudaError_t e = cudaErrorInvalidValue;
     if (c.path == QG_PATH_GEMV) {
-        if (p.op == QG_OP_W4A16)
+        if (p.op == QG_OP_W4A16 && c.bn == 2)
+            e = launch_gemv_w4a16_h2(p, c, d->err_word, stream);
+        else if (p.op == QG_OP_W4A16)
             e = c.stages ? launch_gemv_w4a16_tma(p, c, d->err_word, stream)
                          : launch_gemv_w4a16(p, c, stream);
         else if (p.op == QG_OP_W2A8 && c.stages)
@@ -472,6 +480,19 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                     c.split_k = s;
                     if (supports(p, c)) out.push_back(c);
                 }
+        if (p.op == QG_OP_W4A16 && p.M <= 8) {
+            // 1..8 tokens on the packed fp16 FMA pipe (bn = 2)
+            for (int rows : {32, 64})
+                for (int st : {2, 3, 4, 5, 6})
+                    for (int s = 1; s <= 16; s *= 2) {
+                        c.rows = rows;
+                        c.bn = 2;
+                        c.stages = st;
+                        c.split_k = s;
+                        if (supports(p, c)) out.push_back(c);
+                    }
+            c.bn = 0;
+        }
         if (p.op == QG_OP_W4A16 && p.M == 1) {
             // one token on the FMA pipe (TMA-fed kernel, bn = 1)
             for (int rows : {32, 64, 128})
@@ -635,7 +656,7 @@ qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *
     if (s != QG_OK) return s;
     Problem p = make_problem(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, has_zero);
     qgemm_config_t c = choose(p, split_k, d->sms);
-    if (c.path != QG_PATH_GEMV || c.stages == 0) {   // this form lives in the TMA-fed kernel
+    if (c.path != QG_PATH_GEMV || c.stages == 0 || c.bn == 2) {   // this form lives in the TMA-fed kernel
         std::memset(&c, 0, sizeof(c));
         c.path = QG_PATH_GEMV;
         c.rows = 32;
@@ -844,7 +865,7 @@ qg_status qgemm_w4a16_splitk_f32_noalloc(const void *A, const uint32_t *Wq, cons
     }
     Problem p = make_problem(QG_OP_W4A16, A, Wq, scales, zeros, C, M, N, K, group_size, has_zero);
     qgemm_config_t c = choose(p, split_k, d->sms);
-    if (c.path != QG_PATH_GEMV || c.stages == 0) {
+    if (c.path != QG_PATH_GEMV || c.stages == 0 || c.bn == 2) {
         std::memset(&c, 0, sizeof(c));
         c.path = QG_PATH_GEMV;
         c.rows = 32;
@@ -897,6 +918,14 @@ qg_status qgemm_w2a8(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int
 {
     return matmul(QG_OP_W2A8, A, Wq, nullptr, nullptr, C, M, N, K, group_size, split_k, has_zero,
                   stream);
+}
+
+qg_status qgemm_w2a8_interleaved(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int N,
+                                 int K, int group_size, int split_k, int has_zero,
+                                 cudaStream_t stream)
+{
+    return matmul(QG_OP_W2A8_INTERLEAVED, A, Wq, nullptr, nullptr, C, M, N, K, group_size, split_k,
+                  has_zero, stream);
 }
 
 qg_status qgemm_dense_f16(const void *A, const void *W, void *C, int M, int N, int K,
@@ -955,6 +984,24 @@ qg_status quant_pack_int2(const int8_t *vals, uint32_t *packed, int M, int N, in
     qg_status s = probe_device(&d);
     if (s != QG_OK) return s;
     if (launch_pack_int2(vals, packed, N, K, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+qg_status quant_pack_int2_interleaved(const int8_t *vals, uint32_t *packed, int M, int N, int K,
+                                      int group_size, int split_k, int has_zero,
+                                      cudaStream_t stream)
+{
+    (void)M; (void)group_size; (void)split_k; (void)has_zero;
+    if (!vals || !packed || N <= 0 || K <= 0) return QG_ERR_INVALID_ARG;
+    if (K % 64) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(vals, 16) || !aligned(packed, 16)) return QG_ERR_ALIGNMENT;
+    DeviceInfo *d = nullptr;
+    qg_status s = probe_device(&d);
+    if (s != QG_OK) return s;
+    if (launch_pack_int2_interleaved(vals, packed, N, K, stream) != cudaSuccess) {
         cudaGetLastError();
         return QG_ERR_CUDA;
     }

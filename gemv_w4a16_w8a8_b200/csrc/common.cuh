@@ -22,7 +22,8 @@ struct Problem {
     int M, N, K;
     int gs;        // effective group size (K when the caller passed -1 / 0)
     int has_zero;
-    int interleaved = 0;   // W4A16: 1 = codes of each word in nibble order 0,2,4,6,1,3,5,7
+    int interleaved = 0;   // 1 = the interleaved weight layout (W4A16: nibbles hold codes
+                           // 0,2,4,6,1,3,5,7; W2A8: fields hold 0,4,1,5,2,6,3,7, 8,12,...)
     int sms = 148;         // multiprocessors of the device (persistent grids)
     const float *mult = nullptr;   // W8A8: per-channel multiplier -> int8 output (else int32)
 };
@@ -47,6 +48,10 @@ size_t gemv_w4a16_ws_tiles(const Problem &p, const qgemm_config_t &cfg);
 // Persistent stream-K W4A16 kernel (path QG_PATH_STREAM); C must be zeroed first.
 cudaError_t launch_gemv_w4a16_stream(const Problem &p, const qgemm_config_t &cfg,
                                      unsigned int *err, cudaStream_t stream);
+// W4A16 for 1..8 tokens on the packed fp16 FMA pipe (config: path GEMV, bn = 2).
+cudaError_t launch_gemv_w4a16_h2(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
+                                 cudaStream_t stream);
+int gemv_w4a16_h2_tokens(int M);
 cudaError_t launch_gemv_w2a8_tma(const Problem &p, const qgemm_config_t &cfg, unsigned int *err,
                                  cudaStream_t stream);
 cudaError_t launch_gemv_int(const Problem &p, const qgemm_config_t &cfg, cudaStream_t stream);
@@ -62,12 +67,15 @@ cudaError_t launch_rtn_int4(const __half *W, uint32_t *Wq, __half *S, __half *Z,
                             int gs, cudaStream_t stream);
 cudaError_t launch_pack_int2(const int8_t *vals, uint32_t *packed, int N, int K,
                              cudaStream_t stream);
+cudaError_t launch_pack_int2_interleaved(const int8_t *vals, uint32_t *packed, int N, int K,
+                                         cudaStream_t stream);
 cudaError_t launch_tc(const Problem &p, const qgemm_config_t &cfg, unsigned int *err_word,
                       cudaStream_t stream);
 
 // Whether a configuration can run the problem (tile and alignment rules of its kernel).
 bool gemv_w4a16_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w4a16_tma_supports(const Problem &p, const qgemm_config_t &cfg);
+bool gemv_w4a16_h2_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w4a16_stream_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_w2a8_tma_supports(const Problem &p, const qgemm_config_t &cfg);
 bool gemv_int_supports(const Problem &p, const qgemm_config_t &cfg);
@@ -160,6 +168,13 @@ __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b)
 {
     uint32_t d;
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 

@@ -10,8 +10,9 @@
 // value is u' - 2 and u' is an unsigned 2-bit number. XOR-ing the word with 0xAAAAAAAA forms
 // all sixteen u' at once; (w' >> 2j) & 0x03030303 puts fields j, j+4, j+8, j+12 into the four
 // bytes of one register, which dp4a multiplies (unsigned x signed) against the activations
-// gathered the same way with two rounds of PRMT. The -2 * sum(a) correction is one more dp4a
-// per activation register, shared by all rows of the warp.
+// gathered the same way with two rounds of PRMT (one round for the interleaved layout). The
+// -2 * sum(a) correction is one more dp4a per activation register, shared by all rows of the
+// warp.
 #include "common.cuh"
 
 namespace qg {
@@ -42,8 +43,21 @@ __device__ __forceinline__ void gather_stride4(const uint32_t r0, const uint32_t
     p[3] = prmt(t1, t3, 0x7632);
 }
 
-// R rows per warp, MT tokens per CTA. INT2 selects the packed 2-bit weight format.
-template <int R, int MT, bool INT2>
+// The same for the interleaved int2 layout, whose fields j, j+4, j+8, j+12 hold values
+// (0,2,8,10), (4,6,12,14), (1,3,9,11), (5,7,13,15) for j = 0..3: one round of PRMT.
+__device__ __forceinline__ void gather_interleaved(const uint32_t r0, const uint32_t r1,
+                                                   const uint32_t r2, const uint32_t r3,
+                                                   uint32_t (&p)[4])
+{
+    p[0] = prmt(r0, r2, 0x6420);
+    p[1] = prmt(r1, r3, 0x6420);
+    p[2] = prmt(r0, r2, 0x7531);
+    p[3] = prmt(r1, r3, 0x7531);
+}
+
+// R rows per warp, MT tokens per CTA. INT2 selects the packed 2-bit weight format, ILV its
+// interleaved layout.
+template <int R, int MT, bool INT2, bool ILV = false>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_int_kernel(const int8_t *__restrict__ A, const uint8_t *__restrict__ W,
                 int32_t *__restrict__ C, int M, int N, int K, int chunks_per_split,
@@ -123,7 +137,8 @@ gemv_int_kernel(const int8_t *__restrict__ A, const uint8_t *__restrict__ W,
                     for (int q = 0; q < 4; ++q) {
                         const uint4 a = aok[t] ? ld_cached_v4(arow[t] + (size_t)c * 64 + 16 * q)
                                                : make_uint4(0u, 0u, 0u, 0u);
-                        gather_stride4(a.x, a.y, a.z, a.w, ap[q]);
+                        if constexpr (ILV) gather_interleaved(a.x, a.y, a.z, a.w, ap[q]);
+                        else gather_stride4(a.x, a.y, a.z, a.w, ap[q]);
                         int s = asum[t];
                         s = dp4a_ss(0x01010101, (int)a.x, s);
                         s = dp4a_ss(0x01010101, (int)a.y, s);
@@ -173,7 +188,9 @@ void launch_one(const Problem &p, int split_k, cudaStream_t stream)
     const int cps = (nchunks + split_k - 1) / split_k;
     const int splits = (nchunks + cps - 1) / cps;
     dim3 grid((p.N + kWarps * R - 1) / (kWarps * R), splits, (p.M + MT - 1) / MT);
-    gemv_int_kernel<R, MT, INT2><<<grid, kWarps * 32, 0, stream>>>(
+    auto kern = (INT2 && p.interleaved) ? gemv_int_kernel<R, MT, INT2, true>
+                                        : gemv_int_kernel<R, MT, INT2, false>;
+    kern<<<grid, kWarps * 32, 0, stream>>>(
         static_cast<const int8_t *>(p.A), static_cast<const uint8_t *>(p.W),
         static_cast<int32_t *>(p.C), p.M, p.N, p.K, cps, split_k > 1 ? 1 : 0, p.mult);
 }

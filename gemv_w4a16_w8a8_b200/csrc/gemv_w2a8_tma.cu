@@ -7,7 +7,8 @@
 // Upcast: XOR with 0xAAAAAAAA turns every field u into u' = u ^ 2 (the value is u' - 2, with u'
 // an unsigned 0..3), and (w' >> 2j) & 0x03030303 (j = 0..3) places fields j, j+4, j+8, j+12 in
 // the bytes of one register - 9 instructions for 16 weights. The activations are regathered
-// once per k-block into the same byte order with two rounds of PRMT, and one extra MMA against
+// once per k-block into the same byte order with two rounds of PRMT (one round for the
+// interleaved int2 layout, whose fields hold a different fixed permutation of K), and one extra MMA against
 // an all-ones operand yields sum_k a_k, so that C = sum_k a_k u'_k - 2 sum_k a_k.
 #include <mutex>
 
@@ -39,6 +40,16 @@ __device__ __forceinline__ void gather4(const uint4 &v, uint32_t (&p)[4])
     p[3] = prmt(t1, t3, 0x7632);
 }
 
+// the same for the interleaved layout, whose fields j, j+4, j+8, j+12 hold values (0,2,8,10),
+// (4,6,12,14), (1,3,9,11), (5,7,13,15) for j = 0..3
+__device__ __forceinline__ void gather4_interleaved(const uint4 &v, uint32_t (&p)[4])
+{
+    p[0] = prmt(v.x, v.z, 0x6420);
+    p[1] = prmt(v.y, v.w, 0x6420);
+    p[2] = prmt(v.x, v.z, 0x7531);
+    p[3] = prmt(v.y, v.w, 0x7531);
+}
+
 template <int RB, int NT, int STAGES> struct Layout {
     static constexpr int rows = 16 * RB;
     static constexpr int slot = rows * 64;
@@ -49,7 +60,7 @@ template <int RB, int NT, int STAGES> struct Layout {
     static constexpr int total = ring_bytes + bar_bytes + red_bytes + 16;
 };
 
-template <int RB, int NT, int STAGES>
+template <int RB, int NT, int STAGES, bool ILV>
 __global__ void __launch_bounds__(kWarps * 32)
 gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__restrict__ A,
                      int32_t *__restrict__ C, int M, int N, int K, int kb_per_split,
@@ -131,7 +142,8 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
             for (int q = 0; q < 4; ++q) {
                 uint4 v = make_uint4(0u, 0u, 0u, 0u);
                 if (aok[t]) v = ld_cached_v4(arow[t] + k0 + 16 * q);
-                gather4(v, b[t][q]);
+                if constexpr (ILV) gather4_interleaved(v, b[t][q]);
+                else gather4(v, b[t][q]);
                 mma_16832_u8s8(asum[t], kOnes, b[t][q][0], b[t][q][1]);
                 mma_16832_u8s8(asum2[t], kOnes, b[t][q][2], b[t][q][3]);
             }
@@ -203,11 +215,11 @@ gemv_w2a8_tma_kernel(const __grid_constant__ CUtensorMap tm_w, const int8_t *__r
     }
 }
 
-template <int RB, int NT, int STAGES>
-cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
+template <int RB, int NT, int STAGES, bool ILV>
+cudaError_t launch_layout(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
 {
     using L = Layout<RB, NT, STAGES>;
-    auto kern = gemv_w2a8_tma_kernel<RB, NT, STAGES>;
+    auto kern = gemv_w2a8_tma_kernel<RB, NT, STAGES, ILV>;
     static std::mutex mu;
     static bool opted_in[64] = {};
     int dev = 0;
@@ -233,6 +245,13 @@ cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStr
                                                   static_cast<int32_t *>(p.C), p.M, p.N, p.K,
                                                   kbps, split_k > 1 ? 1 : 0, err);
     return cudaGetLastError();
+}
+
+template <int RB, int NT, int STAGES>
+cudaError_t launch_one(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
+{
+    return p.interleaved ? launch_layout<RB, NT, STAGES, true>(p, split_k, err, stream)
+                         : launch_layout<RB, NT, STAGES, false>(p, split_k, err, stream);
 }
 
 template <int RB, int NT>

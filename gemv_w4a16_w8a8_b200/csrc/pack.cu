@@ -1,5 +1,6 @@
 // Weight packing kernels: uint8 int4 codes -> 8 per uint32, int8 int2 values -> 16 per uint32.
-// Element k of a row lands at bits 4*(k%8) (int4) or 2*(k%16) (int2) of word k/8 (k/16).
+// Element k of a row lands at bits 4*(k%8) (int4) or 2*(k%16) (int2) of word k/8 (k/16); the
+// interleaved layouts permute the elements inside each word (see the kernels).
 // Each thread turns 16 output bytes' worth of input into one 128-bit store.
 #include <algorithm>
 
@@ -70,6 +71,24 @@ __global__ void pack_int2_kernel(const int8_t *__restrict__ vals, uint32_t *__re
             const uint4 a = ld_stream_v4(vals + 64 * u + 16 * q);
             w[q] = fields4(a.x) | (fields4(a.y) << 8) | (fields4(a.z) << 16) |
                    (fields4(a.w) << 24);
+        }
+        reinterpret_cast<uint4 *>(packed)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// interleaved int2 layout: fields 0..15 of a word hold values 0,4,1,5,2,6,3,7, 8,12,9,13,10,14,11,15
+__global__ void pack_int2_interleaved_kernel(const int8_t *__restrict__ vals,
+                                             uint32_t *__restrict__ packed, size_t units)
+{
+    for (size_t u = blockIdx.x * (size_t)blockDim.x + threadIdx.x; u < units;
+         u += (size_t)gridDim.x * blockDim.x) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 a = ld_stream_v4(vals + 64 * u + 16 * q);
+            w[q] = fields4(prmt(a.x, a.y, 0x5140)) | (fields4(prmt(a.x, a.y, 0x7362)) << 8) |
+                   (fields4(prmt(a.z, a.w, 0x5140)) << 16) |
+                   (fields4(prmt(a.z, a.w, 0x7362)) << 24);
         }
         reinterpret_cast<uint4 *>(packed)[u] = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -173,6 +192,14 @@ cudaError_t launch_pack_int2(const int8_t *vals, uint32_t *packed, int N, int K,
 {
     const size_t units = (size_t)N * K / 64;
     pack_int2_kernel<<<grid_for(units), 256, 0, stream>>>(vals, packed, units);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_int2_interleaved(const int8_t *vals, uint32_t *packed, int N, int K,
+                                         cudaStream_t stream)
+{
+    const size_t units = (size_t)N * K / 64;
+    pack_int2_interleaved_kernel<<<grid_for(units), 256, 0, stream>>>(vals, packed, units);
     return cudaGetLastError();
 }
 

@@ -38,9 +38,10 @@
 namespace qg {
 namespace {
 
-enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3, kW4A16I = 4 };   // I: interleaved int4
+enum Mode { kDense = 0, kW8A8 = 1, kW4A16 = 2, kW2A8 = 3, kW4A16I = 4, kW2A8I = 5 };   // I: interleaved
 
 constexpr bool is_w4(int m) { return m == kW4A16 || m == kW4A16I; }
+constexpr bool is_w2(int m) { return m == kW2A8 || m == kW2A8I; }
 
 constexpr int kThreads = 512;
 constexpr int kRowsW = 128;            // weight rows per tile (MMA M)
@@ -105,13 +106,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
 template <int MODE, int BN>
 __host__ __device__ constexpr uint32_t instr_desc()
 {
-    constexpr bool i8 = (MODE == kW8A8 || MODE == kW2A8);
+    constexpr bool i8 = (MODE == kW8A8 || is_w2(MODE));
     return (i8 ? 2u : 1u) << 4 | (i8 ? 1u : 0u) << 7 | (i8 ? 1u : 0u) << 10 |
            (uint32_t)(BN >> 3) << 17 | (uint32_t)(kRowsW >> 4) << 24;
 }
 
 template <int MODE> struct Traits {
-    static constexpr bool packed = (is_w4(MODE) || MODE == kW2A8);
+    static constexpr bool packed = (is_w4(MODE) || is_w2(MODE));
     static constexpr int w_tma_bytes = packed ? kRowsW * 32 : kRowsW * kSlabBytes;
     static constexpr int w_mma_bytes = packed ? kRowsW * kSlabBytes : 0;   // dequant target
     static constexpr int k_per_slab = (MODE == kDense || is_w4(MODE)) ? 64 : 128;
@@ -234,30 +235,34 @@ __device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, 
 }
 
 // Upcast half a slab of packed int2 (p = words 4h..4h+3 of weight row r: 64 values) into int8.
+// Byte-table lookup: PRMT with both sources holding the int8 values of the four 2-bit codes
+// (0, 1, -2, -1 -> 0x00, 0x01, 0xFE, 0xFF) turns the low three bits of each selector nibble into
+// a byte (bit 2 picks the second, identical copy of the table), so (w >> s) & 0x7777 for
+// s = 0, 2, 16, 18 gives the values of fields (0,2,4,6), (1,3,5,7), (8,10,12,14), (9,11,13,15).
+// In the interleaved layout those are values 0-3, 4-7, 8-11, 12-15 in K order (11 instructions
+// a word); the natural layout needs one more byte transpose of register pairs (15).
+template <bool ILV>
 __device__ __forceinline__ void dequant_w2(const uint4 &p, uint8_t *dst, int r, int h)
 {
+    constexpr uint32_t kTable = 0xFFFE0100u, kSel = 0x7777u;
     const uint32_t words[4] = {p.x, p.y, p.z, p.w};
     uint8_t *row = dst + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const uint32_t wf = words[j] ^ 0xAAAAAAAAu;           // u' = u ^ 2, value = u' - 2
-        const uint32_t f0 = wf & 0x03030303u;                 // fields 0, 4, 8, 12
-        const uint32_t f1 = (wf >> 2) & 0x03030303u;          // fields 1, 5, 9, 13
-        const uint32_t f2 = (wf >> 4) & 0x03030303u;
-        const uint32_t f3 = (wf >> 6) & 0x03030303u;
-        // 4x4 byte transpose -> natural order (fields 4i .. 4i+3 in register i)
-        const uint32_t t0 = prmt(f0, f1, 0x5140), t1 = prmt(f0, f1, 0x7362);
-        const uint32_t t2 = prmt(f2, f3, 0x5140), t3 = prmt(f2, f3, 0x7362);
+        const uint32_t w = words[j];
+        const uint32_t d0 = prmt(kTable, kTable, w & kSel);
+        const uint32_t d1 = prmt(kTable, kTable, (w >> 2) & kSel);
+        const uint32_t d2 = prmt(kTable, kTable, (w >> 16) & kSel);
+        const uint32_t d3 = prmt(kTable, kTable, (w >> 18) & kSel);
         uint4 o;
-        o.x = prmt(t0, t2, 0x5410);
-        o.y = prmt(t0, t2, 0x7632);
-        o.z = prmt(t1, t3, 0x5410);
-        o.w = prmt(t1, t3, 0x7632);
-        // per byte: (u' + 0x7E) ^ 0x80 = u' - 2 (no carry leaves a byte: u' + 0x7E <= 0x81)
-        o.x = (o.x + 0x7E7E7E7Eu) ^ 0x80808080u;
-        o.y = (o.y + 0x7E7E7E7Eu) ^ 0x80808080u;
-        o.z = (o.z + 0x7E7E7E7Eu) ^ 0x80808080u;
-        o.w = (o.w + 0x7E7E7E7Eu) ^ 0x80808080u;
+        if constexpr (ILV) {
+            o = make_uint4(d0, d1, d2, d3);
+        } else {
+            o.x = prmt(d0, d1, 0x5140);   // values 0, 1, 2, 3
+            o.y = prmt(d0, d1, 0x7362);   // 4 .. 7
+            o.z = prmt(d2, d3, 0x5140);   // 8 .. 11
+            o.w = prmt(d2, d3, 0x7362);   // 12 .. 15
+        }
         *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }
 }
@@ -701,7 +706,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                             dequant_w4<MODE == kW4A16I>(pk[j][x], w_dq(d), r, TOKA ? x : h, sc2[j],
                                                         nz2[j]);
                         else
-                            dequant_w2(pk[j][x], w_dq(d), r, h);
+                            dequant_w2<MODE == kW2A8I>(pk[j][x], w_dq(d), r, h);
                     }
                     if constexpr (per_slab_handoff(BN)) {
                         // this slab's upcast stores become visible to the tensor core (async
@@ -969,7 +974,7 @@ template <int MODE, int BN>
 cudaError_t launch_stages(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                           cudaStream_t stream)
 {
-    if constexpr (is_w4(MODE) || MODE == kW2A8)
+    if constexpr (is_w4(MODE) || is_w2(MODE))
         if (packed_group(p, BN, c.stages) == 4) return launch_stages_pg<MODE, BN, 4>(p, c, err, stream);
     return launch_stages_pg<MODE, BN, 1>(p, c, err, stream);
 }
@@ -1070,7 +1075,9 @@ cudaError_t launch_tc(const Problem &p, const qgemm_config_t &c, unsigned int *e
     case kW4A16:
         return p.interleaved ? launch_bn<kW4A16I>(p, c, err, stream)
                              : launch_bn<kW4A16>(p, c, err, stream);
-    default: return launch_bn<kW2A8>(p, c, err, stream);
+    default:
+        return p.interleaved ? launch_bn<kW2A8I>(p, c, err, stream)
+                             : launch_bn<kW2A8>(p, c, err, stream);
     }
 }
 

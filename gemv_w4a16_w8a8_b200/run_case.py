@@ -39,6 +39,8 @@ def main(argv=None) -> int:
     ap.add_argument("--swap-ab", type=int, default=-1,
                     help="TC: 1 = weights in the MMA's M side, 0 = token-major tile")
     ap.add_argument("--copies", type=int, default=0, help="weight copies (0: >= 3x L2)")
+    ap.add_argument("--interleaved", action="store_true",
+                    help="w4a16 / w2a8: weights in the interleaved (pre-shuffled) layout")
     a = ap.parse_args(argv)
 
     dev = torch.device("cuda", 0)
@@ -46,15 +48,20 @@ def main(argv=None) -> int:
     up = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
     opc = {"w4a16": qg.OP_W4A16, "w8a8": qg.OP_W8A8, "w2a8": qg.OP_W2A8,
            "dense": qg.OP_DENSE_F16}[a.op]
+    ilv = a.interleaved and a.op in ("w4a16", "w2a8")
+    if ilv:
+        opc = qg.OP_W4A16_INTERLEAVED if a.op == "w4a16" else qg.OP_W2A8_INTERLEAVED
     gs = a.gs if a.op == "w4a16" else -1
     hz = a.has_zero if a.op == "w4a16" else 0
     if a.op == "w4a16":
         d = synth.w4a16_inputs(M, N, K, gs, bool(hz), seed=0)
-        A, W = up(d["A"]), qg.quant_pack_int4(up(d["codes"]))
+        pack = qg.quant_pack_int4_interleaved if ilv else qg.quant_pack_int4
+        mm = qg.qgemm_w4a16_interleaved if ilv else qg.qgemm_w4a16
+        A, W = up(d["A"]), pack(up(d["codes"]))
         S = up(d["scales"])
         Z = up(d["zeros"]) if hz else None
         wbytes = N * K // 2
-        run = lambda w, C: qg.qgemm_w4a16(A, w, S, Z, C=C, group_size=gs, split_k=a.split_k)
+        run = lambda w, C: mm(A, w, S, Z, C=C, group_size=gs, split_k=a.split_k)
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + N * (K // (K if gs <= 0 else gs)) * 2 * (1 + hz) + 2 * M * K + 2 * M * N
     elif a.op == "w8a8":
@@ -66,9 +73,11 @@ def main(argv=None) -> int:
         nbytes = wbytes + M * K + 4 * M * N
     elif a.op == "w2a8":
         d = synth.w2a8_inputs(M, N, K, seed=0)
-        A, W = up(d["A"]), qg.quant_pack_int2(up(d["Wv"]))
+        pack = qg.quant_pack_int2_interleaved if ilv else qg.quant_pack_int2
+        mm = qg.qgemm_w2a8_interleaved if ilv else qg.qgemm_w2a8
+        A, W = up(d["A"]), pack(up(d["Wv"]))
         wbytes = N * K // 4
-        run = lambda w, C: qg.qgemm_w2a8(A, w, C=C, split_k=a.split_k)
+        run = lambda w, C: mm(A, w, C=C, split_k=a.split_k)
         C = torch.empty((M, N), dtype=torch.int32, device=dev)
         nbytes = wbytes + M * K + 4 * M * N
     else:

@@ -66,7 +66,8 @@ typedef enum qg_op {
     QG_OP_W8A8 = 1,
     QG_OP_W2A8 = 2,
     QG_OP_DENSE_F16 = 3,
-    QG_OP_W4A16_INTERLEAVED = 4   /* W4A16 with weights from quant_pack_int4_interleaved */
+    QG_OP_W4A16_INTERLEAVED = 4,  /* W4A16 with weights from quant_pack_int4_interleaved */
+    QG_OP_W2A8_INTERLEAVED = 5    /* W2A8 with weights from quant_pack_int2_interleaved  */
 } qg_op;
 
 typedef enum qg_path {
@@ -235,6 +236,22 @@ qg_status qgemm_w2a8(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int
                      int group_size, int split_k, int has_zero, cudaStream_t stream);
 
 /*
+ * W2A8 with weights in the interleaved (pre-shuffled) layout that quant_pack_int2_interleaved
+ * writes: within each uint32 word the values k = 16j .. 16j+15 sit in 2-bit fields
+ * 0, 2, 4, 6, 1, 3, 5, 7, 8, 10, 12, 14, 9, 11, 13, 15 (fields 0..15 hold values 0, 4, 1, 5, 2,
+ * 6, 3, 7, 8, 12, 9, 13, 10, 14, 11, 15), so that the tensor-core path's upcast (a byte-table
+ * PRMT on the low 3 bits of each nibble of w, w >> 2, w >> 16 and w >> 18) yields four int8
+ * registers already in K order, with no byte transpose. pytorch/ao issue #2752 ("Migrating from
+ * AffineQuantizedTensor + Layouts to tensor subclasses"), packing-format list: pre-shuffled
+ * layouts that move the permutation out of the hot loop. Result and every other argument as
+ * qgemm_w2a8 on the naturally packed weights of the same values (exact, bit-identical).
+ * Configurations are kept under QG_OP_W2A8_INTERLEAVED.
+ */
+qg_status qgemm_w2a8_interleaved(const int8_t *A, const uint32_t *Wq, int32_t *C, int M, int N,
+                                 int K, int group_size, int split_k, int has_zero,
+                                 cudaStream_t stream);
+
+/*
  * Dense fp16 baseline. A: fp16 [M, K]; W: fp16 [N, K]; C: fp16 [M, N] = A . W^T with fp32
  * accumulation. Requires K % 8 == 0.
  */
@@ -287,6 +304,17 @@ qg_status quant_pack_int4_interleaved(const uint8_t *codes, uint32_t *packed, in
  */
 qg_status quant_pack_int2(const int8_t *vals, uint32_t *packed, int M, int N, int K,
                           int group_size, int split_k, int has_zero, cudaStream_t stream);
+
+/*
+ * vals: int8 [N, K] holding values -2..1 (only the low 2 bits are used) -> packed: uint32
+ * [N, K/16] in the interleaved layout of qgemm_w2a8_interleaved:
+ *     packed[n, j] = sum_i (vals[n, 16j+i] & 3) << 2 * pos(i),
+ *     pos(i) = 8 * (i / 8) + 2 * (i % 4) + (i % 8) / 4.
+ * Requires K % 64 == 0. Other arguments as quant_pack_int2.
+ */
+qg_status quant_pack_int2_interleaved(const int8_t *vals, uint32_t *packed, int M, int N, int K,
+                                      int group_size, int split_k, int has_zero,
+                                      cudaStream_t stream);
 
 /* ---- configuration ---------------------------------------------------------------------------- */
 

@@ -304,3 +304,20 @@ def test_selftest_limit_validated_before_the_device():
     L = qg.lib()
     assert L.qgemm_selftest_bounded_wait(0, None) == qg.QG_ERR_INVALID_ARG
     assert L.qgemm_selftest_bounded_wait(2000001, None) == qg.QG_ERR_INVALID_ARG
+
+
+def test_half2_gemv_config_rules():
+    """Path GEMV with bn = 2 (packed fp16 FMA pipe): 1..8 tokens, 32 or 64 rows, 2..6 stages,
+    group sizes that are multiples of 128; the fp32-workspace split-K form ignores it."""
+    ok = {"path": qg.PATH_GEMV, "rows": 64, "bm": 0, "bn": 2, "bk": 0, "stages": 4, "split_k": 2,
+          "swap_ab": 0}
+    for M in (1, 2, 3, 4, 8):
+        qg.qgemm_set_config(qg.OP_W4A16, M, 4096, 4096, 128, 1, ok)
+        assert qg.qgemm_plan(qg.OP_W4A16, M, 4096, 4096, 128, 1)["bn"] == 2
+        qg.qgemm_set_config(qg.OP_W4A16, M, 4096, 4096, 128, 1, None)
+    for bad in ({"rows": 16}, {"rows": 128}, {"stages": 1}, {"stages": 7}, {"split_k": 65}):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, 1, 4096, 4096, 128, 1, {**ok, **bad})
+    for M, gs in ((9, 128), (1, 64), (1, 32)):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, M, 4096, 4096, gs, 1, ok)
