@@ -90,6 +90,84 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
                  : "memory");
 }
 
+// ---- CTA pairs (cta_group::2): one MMA spans the tensor cores of two SMs of a cluster --------
+// The leader (rank 0) issues every MMA; A's 256 rows are the two CTAs' 128-row weight slabs and
+// B's N rows the two CTAs' halves of the token tile, each read from its own CTA's shared memory
+// at the same offset; each CTA's TMEM holds the accumulator rows of its own weight rows.
+
+template <int MODE>
+__device__ __forceinline__ void mma_issue_pair(uint32_t dtm, uint64_t a, uint64_t b, uint32_t idesc,
+                                               uint32_t accumulate)
+{
+    if constexpr (MODE == kDense || is_w4(MODE)) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtm),
+                     "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+                     : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtm),
+                     "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+                     : "memory");
+    }
+}
+
+// arrive on the barrier at the same offset in both CTAs of the pair once the MMAs finish
+__device__ __forceinline__ void mma_commit_pair_both(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::"
+                 "cluster.b64 [%0], %1;" ::"r"(bar), "h"((uint16_t)3)
+                 : "memory");
+}
+
+// arrive on this CTA's own barrier once the MMAs finish
+__device__ __forceinline__ void mma_commit_pair_local(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// address of the same shared-memory location in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// arrival (release at cluster scope) on a barrier given by its shared::cluster address
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// every thread of both CTAs
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+// 2-D TMA load into this CTA's shared memory that completes its bytes on a barrier of either
+// CTA of the pair (given by its shared::cluster address); no multicast
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map,
+                                                 uint32_t bar_cluster, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx"
+                 "::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
 {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -101,14 +179,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Instruction descriptor: dense, K-major A and B, M = 128, N = BN.
+// Instruction descriptor: dense, K-major A and B, M = MR (128, or 256 for a CTA pair), N = BN.
 //   fp16 x fp16 -> fp32: D format 1, A/B format 0.   int8 x int8 -> int32: D 2, A/B 1 (signed).
-template <int MODE, int BN>
+template <int MODE, int BN, int MR = kRowsW>
 __host__ __device__ constexpr uint32_t instr_desc()
 {
     constexpr bool i8 = (MODE == kW8A8 || is_w2(MODE));
     return (i8 ? 2u : 1u) << 4 | (i8 ? 1u : 0u) << 7 | (i8 ? 1u : 0u) << 10 |
-           (uint32_t)(BN >> 3) << 17 | (uint32_t)(kRowsW >> 4) << 24;
+           (uint32_t)(BN >> 3) << 17 | (uint32_t)(MR >> 4) << 24;
 }
 
 template <int MODE> struct Traits {
@@ -144,47 +222,53 @@ constexpr int kSinkBytes = 256 * 4;
 constexpr int min_dq(int pg, int bn) { return (pg < 2 || per_slab_handoff(bn)) ? 2 : pg; }
 constexpr int want_dq(int pg, int bn) { return per_slab_handoff(bn) ? 3 : min_dq(pg, bn); }
 
-constexpr int smem_total(bool packed, int bn, int stages, int dq, int pg, int sp, int wr = kRowsW)
+// ar: activation rows of a stage held by this CTA (the MMA's N, or half of it for a CTA pair)
+constexpr int smem_total(bool packed, int ar, int stages, int dq, int pg, int sp, int wr = kRowsW)
 {
-    return packed ? 1024 + stages * bn * kSlabBytes + sp * wr * 32 * pg + dq * wr * kSlabBytes +
+    return packed ? 1024 + stages * ar * kSlabBytes + sp * wr * 32 * pg + dq * wr * kSlabBytes +
                         kSinkBytes + 8 * (2 * stages + 2 * sp + 2 * dq + 5) + 16
-                  : 1024 + stages * (kRowsW * kSlabBytes + bn * kSlabBytes) + 8 * (2 * stages + 5) +
+                  : 1024 + stages * (kRowsW * kSlabBytes + ar * kSlabBytes) + 8 * (2 * stages + 5) +
                         16;
 }
 
 // Packed-weight copies in flight: 12 single slabs, or 6 / 4 grouped copies; for token tiles of
 // 128 and more, fewer when a deep activation ring would otherwise leave less than want_dq upcast
 // buffers (one grouped copy holds 4 slabs, so 2-3 copies already run far ahead of the MMA).
-constexpr int packed_stages(int pg, int bn, int stages, int wr = kRowsW)
+constexpr int packed_stages(int pg, int bn, int stages, int wr = kRowsW, int ar = 0)
 {
     if (pg == 1) return 12;
     if (bn <= 64) return 6;
+    const int a = ar ? ar : bn;
     int sp = 4;
-    while (sp > 2 && smem_total(true, bn, stages, want_dq(pg, bn), pg, sp, wr) > kMaxSmem) --sp;
+    while (sp > 2 && smem_total(true, a, stages, want_dq(pg, bn), pg, sp, wr) > kMaxSmem) --sp;
     return sp;
 }
 
 // Upcast-weight buffers: as many as fit, up to 8. Each buffer makes a round trip (upcast, fence,
 // arrive, MMA, commit, release) whose latency bounds the throughput when the token tile is small,
 // so small tiles take the most. A plan below min_dq is reported as not fitting (smem_bytes).
-constexpr int dq_buffers(bool packed, int bn, int stages, int pg, int wr = kRowsW)
+constexpr int dq_buffers(bool packed, int bn, int stages, int pg, int wr = kRowsW, int ar = 0)
 {
     if (!packed) return 0;
-    const int sp = packed_stages(pg, bn, stages, wr);
+    const int a = ar ? ar : bn;
+    const int sp = packed_stages(pg, bn, stages, wr, a);
     int d = 8;
-    while (d > min_dq(pg, bn) && smem_total(true, bn, stages, d, pg, sp, wr) > kMaxSmem) --d;
+    while (d > min_dq(pg, bn) && smem_total(true, a, stages, d, pg, sp, wr) > kMaxSmem) --d;
     return d;
 }
 
-// BN: tokens per tile (the MMA's N, or its M in the token-major variant); WR weight rows.
-template <int MODE, int BN, int STAGES, int PG, bool TOKA = false> struct Smem {
+// BN: tokens per tile (the MMA's N, or its M in the token-major variant); WR weight rows of this
+// CTA. PAIR: a CTA pair shares each MMA (cta_group::2), and each CTA holds half of the tile's
+// tokens (AR rows of every activation stage).
+template <int MODE, int BN, int STAGES, int PG, bool TOKA = false, bool PAIR = false> struct Smem {
     static constexpr bool packed = Traits<MODE>::packed;
     static constexpr int WR = wrows<TOKA>();
-    static constexpr int a_bytes = BN * kSlabBytes;
+    static constexpr int AR = PAIR ? BN / 2 : BN;
+    static constexpr int a_bytes = AR * kSlabBytes;
     static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
     static constexpr int pw_bytes = WR * 32 * PG;                // packed weight copy (PG slabs)
-    static constexpr int sp = packed ? packed_stages(PG, BN, STAGES, WR) : 0;
-    static constexpr int dq = dq_buffers(packed, BN, STAGES, PG, WR);
+    static constexpr int sp = packed ? packed_stages(PG, BN, STAGES, WR, AR) : 0;
+    static constexpr int dq = dq_buffers(packed, BN, STAGES, PG, WR, AR);
     static constexpr int dq_bytes = WR * kSlabBytes;
     // byte offsets from the 1024-aligned base
     static constexpr int ring_bytes = packed ? STAGES * a_bytes : STAGES * (w_bytes + a_bytes);
@@ -193,7 +277,7 @@ template <int MODE, int BN, int STAGES, int PG, bool TOKA = false> struct Smem {
     static constexpr int sink_off = dq_off + dq * dq_bytes;
     static constexpr int bar_off = sink_off + (packed ? kSinkBytes : 0);
     static constexpr int nbars = 2 * STAGES + 2 * sp + 2 * dq + 5;
-    static constexpr int total = smem_total(packed, BN, STAGES, dq, PG, sp, WR);
+    static constexpr int total = smem_total(packed, AR, STAGES, dq, PG, sp, WR);
 };
 
 // two accumulator buffers of BN fp32 / int32 columns (the allocation is a power of two >= 32)
@@ -307,7 +391,7 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
 //              in the token-major variant)
 // TOKA: token-major variant (W4A16): tiles of kTokT = BN tokens x kRowsT weight rows, tokens in
 // the MMA's M, weights in its N; the accumulator holds one token per TMEM lane.
-template <int MODE, int BN, int STAGES, int PG, bool TOKA>
+template <int MODE, int BN, int STAGES, int PG, bool TOKA, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                const __half *__restrict__ S, const __half *__restrict__ Z, void *__restrict__ C,
@@ -315,12 +399,21 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                const float *__restrict__ mult, unsigned int *err)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES, PG, TOKA>;
+    using L = Smem<MODE, BN, STAGES, PG, TOKA, PAIR>;
     static_assert(!TOKA || (is_w4(MODE) && BN == kTokT), "token-major tiles: W4A16, 128 tokens");
+    static_assert(!PAIR || (!TOKA && BN >= 128), "CTA pairs: weight-major tiles of 128+ tokens");
     constexpr int WR = L::WR;
     constexpr int NMMA = TOKA ? kRowsT : BN;          // the MMA's N (accumulator columns)
     constexpr uint32_t kCols = tmem_cols<NMMA>();
-    constexpr uint32_t kIdesc = instr_desc<MODE, NMMA>();
+    constexpr uint32_t kIdesc = instr_desc<MODE, NMMA, PAIR ? 2 * kRowsW : kRowsW>();
+    // CTA pairs: a unit covers UR = 256 weight rows, this CTA's 128 start at roff, and this CTA
+    // loads tokens aoff .. aoff + AR - 1 of the tile; both CTAs walk the same units
+    constexpr int UR = PAIR ? 2 * kRowsW : WR;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
+    const int roff = PAIR ? (int)rank * kRowsW : 0;
+    const int aoff = PAIR ? (int)rank * L::AR : 0;
+    const int ustart = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int ustep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
@@ -332,7 +425,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int n_tiles = (N + WR - 1) / WR;
+    const int n_tiles = (N + UR - 1) / UR;
     const int t_tiles = (M + BN - 1) / BN;
     const int nkb = (K + T::k_per_slab - 1) / T::k_per_slab;
 
@@ -365,13 +458,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             mbar_init(pfull_bar(p), 1);
             mbar_init(pempty_bar(p), 8);
         }
+        // a pair's leader hears the upcast and epilogue warps of both CTAs
         for (int d = 0; d < DQ; ++d) {
-            mbar_init(dqf_bar(d), 8);
+            mbar_init(dqf_bar(d), PAIR ? 16 : 8);
             mbar_init(dqe_bar(d), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(accf_bar(b), 1);
-            mbar_init(acce_bar(b), 4);
+            mbar_init(acce_bar(b), PAIR ? 8 : 4);
         }
         mbar_init(final_bar, 1);
         *abort_flag = 0;
@@ -379,14 +473,25 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         fence_proxy_async_smem();
     }
     if (warp == 5) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_holder)),
-                     "r"(kCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (PAIR) {
+            // both CTAs of the pair, from the same warp, into the same shared-memory offset
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_holder)),
+                         "r"(kCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_u32(tmem_holder)),
+                         "r"(kCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    // a pair's barriers must be initialised before the other CTA signals them
+    if constexpr (PAIR) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -400,8 +505,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         constexpr uint32_t kTx = L::packed ? L::a_bytes : L::w_bytes + L::a_bytes;
         int it = 0;
         bool stop = false;
-        for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+        for (int u = ustart; u < units && !stop; u += ustep) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
             for (int i = 0; i < w.nk; ++i, ++it) {
                 const int s = it % STAGES;
                 if (!warp_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
@@ -410,26 +515,43 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 }
                 const int kx = (w.kb0 + i) * T::k_per_slab;
                 if (lane == 0) {
-                    mbar_expect_tx(full_bar(s), kTx);
-                    if constexpr (!L::packed)
-                        tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kx, w.n0);
-                    tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kx, w.t0);
+                    if constexpr (PAIR) {
+                        // both CTAs' copies complete on the leader's barrier, which expects both
+                        const uint32_t fb = map_to_rank(full_bar(s), 0);
+                        if (rank == 0) mbar_expect_tx(full_bar(s), 2 * kTx);
+                        if constexpr (!L::packed)
+                            tma_load_2d_pair(smem_u32(w_tma(s)), &tm_w, fb, kx, w.n0 + roff);
+                        tma_load_2d_pair(smem_u32(a_tile(s)), &tm_a, fb, kx, w.t0 + aoff);
+                    } else {
+                        mbar_expect_tx(full_bar(s), kTx);
+                        if constexpr (!L::packed)
+                            tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kx, w.n0);
+                        tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kx, w.t0);
+                    }
                 }
                 __syncwarp();
             }
         }
         // every copy this warp started must land before the CTA can exit
-        for (int i = max(0, it - STAGES); i < it; ++i) {
-            int dummy_abort = 0;
-            mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+        if (!PAIR || rank == 0) {
+            for (int i = max(0, it - STAGES); i < it; ++i) {
+                int dummy_abort = 0;
+                mbar_wait(full_bar(i % STAGES), (i / STAGES) & 1, &dummy_abort, nullptr);
+            }
+        } else if (*abort_flag) {
+            // the second CTA's copies complete on the leader's barrier, which it cannot watch:
+            // after a give-up (the only way it can stop early) it waits 100 us, far beyond the
+            // latency of a copy, before it heads for the exit
+            const uint64_t t0 = global_ns();
+            while (global_ns() - t0 < 100000ull) __nanosleep(1000);
         }
     } else if (warp == 6) {
         if constexpr (L::packed) {
             // ---------------- TMA producer (packed weight slabs) ----------------
             int it = 0;
             bool stop = false;
-            for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+            for (int u = ustart; u < units && !stop; u += ustep) {
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
                 // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
                 for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
@@ -440,7 +562,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     if (lane == 0) {
                         mbar_expect_tx(pfull_bar(p), L::pw_bytes);
                         tma_load_2d(smem_u32(pw_tile(p)), &tm_w, pfull_bar(p), (w.kb0 + i) * 8,
-                                    w.n0);
+                                    w.n0 + roff);
                     }
                     __syncwarp();
                 }
@@ -450,13 +572,13 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 mbar_wait(pfull_bar(i % SP), (i / SP) & 1, &dummy_abort, nullptr);
             }
         }
-    } else if (warp == 5) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 5 && (!PAIR || rank == 0)) {
+        // ---------------- MMA issuer (a pair's leader issues for both CTAs) ----------------
         // Lane 0 issues the MMAs and the commits: a commit tracks the MMAs its own thread issued.
         int it = 0, j = 0;
         bool stop = false;
-        for (int u = blockIdx.x; u < units && !stop; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+        for (int u = ustart; u < units && !stop; u += ustep) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
             if (w.nk == 0) continue;
             const int b = j & 1;
             if (!warp_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
@@ -481,22 +603,38 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 const uint64_t tdesc = sw128_desc(smem_u32(a_tile(s)));
                 const uint64_t adesc = TOKA ? tdesc : wdesc, bdesc = TOKA ? wdesc : tdesc;
                 if (lane == 0) {
+                    if constexpr (PAIR) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
-                        mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
-                                        (i | k) != 0 ? 1u : 0u);
-                    mma_commit(empty_bar(s));
-                    if constexpr (T::packed) mma_commit(dqe_bar(d));
+                        for (int k = 0; k < 4; ++k)
+                            mma_issue_pair<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                                 (i | k) != 0 ? 1u : 0u);
+                        // the slab's buffers go back to their producers in both CTAs
+                        mma_commit_pair_both(empty_bar(s));
+                        if constexpr (T::packed) mma_commit_pair_both(dqe_bar(d));
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)   // 4 MMAs of 32 bytes of K each
+                            mma_issue<MODE>(dtm, adesc + 2 * k, bdesc + 2 * k, kIdesc,
+                                            (i | k) != 0 ? 1u : 0u);
+                        mma_commit(empty_bar(s));
+                        if constexpr (T::packed) mma_commit(dqe_bar(d));
+                    }
                 }
                 __syncwarp();
             }
             if (stop) break;
-            if (lane == 0) mma_commit(accf_bar(b));
+            if (lane == 0) {
+                if constexpr (PAIR) mma_commit_pair_both(accf_bar(b));
+                else mma_commit(accf_bar(b));
+            }
             __syncwarp();
             ++j;
         }
         // nothing may still run on the tensor cores when TMEM is released
-        if (lane == 0) mma_commit(final_bar);
+        if (lane == 0) {
+            if constexpr (PAIR) mma_commit_pair_local(final_bar);
+            else mma_commit(final_bar);
+        }
         __syncwarp();
         int dummy_abort = 0;
         mbar_wait(final_bar, 0, &dummy_abort, nullptr);
@@ -520,12 +658,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             };
             auto settle = [&](Cursor &c) {
                 while (c.u < units && c.i >= c.w.nk) {
-                    c.u += gridDim.x;
+                    c.u += ustep;
                     c.i = 0;
-                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
                 }
             };
-            Cursor cur{(int)blockIdx.x, 0, unit_of(blockIdx.x, n_tiles, t_tiles, BN, nkb, kb_per_split, WR)};
+            Cursor cur{ustart, 0, unit_of(ustart, n_tiles, t_tiles, BN, nkb, kb_per_split, UR)};
             settle(cur);
             // Scales and zeros. Per slab a thread needs s[n][g] and z[n][g] of its row n. Loading
             // those 2-byte values one slab at a time makes every warp touch 32 rows (32 sectors)
@@ -551,24 +689,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 wnd.u = u;
                 wnd.gb = gb;
                 if (u >= units) return;
-                const size_t off = (size_t)min(w.n0 + r, N - 1) * G + gb;
+                const size_t off = (size_t)min(w.n0 + roff + r, N - 1) * G + gb;
                 wnd.s = ld_cached_v4(S + off);
                 wnd.z = Z ? ld_cached_v4(Z + off) : make_uint4(0u, 0u, 0u, 0u);
             };
             // the window after wnd in this CTA's walk (same unit, or the next unit's first one)
             auto next_window = [&](Window &out, const Window &wnd) {
-                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
                 const int g_last = min(((w.kb0 + w.nk) * 64 - 1) / gs, G - 1);
                 if (wnd.gb + 8 <= g_last) {
                     load_window(out, wnd.u, w, wnd.gb + 8);
                     return;
                 }
-                int u = wnd.u + gridDim.x;
+                int u = wnd.u + ustep;
                 Unit nw = w;
                 while (u < units) {
-                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
                     if (nw.nk > 0) break;
-                    u += gridDim.x;
+                    u += ustep;
                 }
                 load_window(out, u, nw, (min((nw.kb0 * 64) / gs, G - 1)) & ~7);
             };
@@ -609,7 +747,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     z_out = 0.f;
                     return;
                 }
-                const int n = min(c.w.n0 + r, N - 1);
+                const int n = min(c.w.n0 + roff + r, N - 1);
                 const int g = group_of(c);
                 s_out = half_bits_to_float(ld_cached_u16(S + (size_t)n * G + g));
                 z_out = Z ? half_bits_to_float(ld_cached_u16(Z + (size_t)n * G + g)) : 0.f;
@@ -710,10 +848,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     }
                     if constexpr (per_slab_handoff(BN)) {
                         // this slab's upcast stores become visible to the tensor core (async
-                        // proxy), then one arrival per warp hands the buffer over
+                        // proxy), then one arrival per warp hands the buffer over (to the
+                        // pair's leader, which issues the MMA)
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(dqf_bar(d));
+                        if (lane == 0) {
+                            if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(dqf_bar(d), 0));
+                            else mbar_arrive(dqf_bar(d));
+                        }
                     }
                 }
                 if (!ok) break;
@@ -723,7 +865,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     __syncwarp();
                     if (lane == 0)
 #pragma unroll
-                        for (int j = 0; j < PG; ++j) mbar_arrive(dqf_bar((it + j) % DQ));
+                        for (int j = 0; j < PG; ++j) {
+                            if constexpr (PAIR)
+                                mbar_arrive_cluster(map_to_rank(dqf_bar((it + j) % DQ), 0));
+                            else
+                                mbar_arrive(dqf_bar((it + j) % DQ));
+                        }
                 }
                 it += PG;
                 ++cur.i;
@@ -735,8 +882,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         const int r = tid;                                 // weight row of the tile = TMEM lane
         const bool pairs = (N & 1) == 0;
         int j = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, WR);
+        for (int u = ustart; u < units; u += ustep) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
             if (w.nk == 0) continue;
             const int b = j & 1;
             bool ok = mbar_wait(accf_bar(b), (j >> 1) & 1, abort_flag, err);
@@ -788,7 +935,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     }
                 }
             } else {
-                const int n = w.n0 + r;
+                const int n = w.n0 + roff + r;
                 // int8 requantisation (int32 modes): this lane's output-channel multiplier
                 const float rq = (T::c_bytes == 4 && mult && n < N) ? mult[n] : 0.f;
                 const uint32_t lane_addr =
@@ -826,21 +973,32 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     }
                 }
             }
-            // this warp is done with accumulator buffer b
+            // this warp is done with accumulator buffer b (the pair's leader waits for both CTAs)
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(b));
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(acce_bar(b), 0));
+                else mbar_arrive(acce_bar(b));
+            }
             ++j;
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    // a pair: the leader's last MMA (waited for above) read the other CTA's shared memory and
+    // wrote its TMEM, so neither CTA releases anything before both are here
+    if constexpr (PAIR) cluster_sync();
+    else __syncthreads();
     if (warp == 5) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kCols)
-                     : "memory");
+        if constexpr (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                         "r"(kCols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                         "r"(kCols)
+                         : "memory");
     }
 }
 
@@ -856,31 +1014,33 @@ int mode_of(int op)
     }
 }
 
-int smem_bytes(int mode, int bn, int stages, int pg, int wr = kRowsW)
+// pair: a CTA pair shares the tile (each CTA holds half of the token rows of a stage)
+int smem_bytes(int mode, int bn, int stages, int pg, int wr = kRowsW, bool pair = false)
 {
     const bool packed = (is_w4(mode) || mode == kW2A8);
-    return smem_total(packed, bn, stages, dq_buffers(packed, bn, stages, pg, wr), pg,
-                      packed ? packed_stages(pg, bn, stages, wr) : 0, wr);
+    const int ar = pair ? bn / 2 : bn;
+    return smem_total(packed, ar, stages, dq_buffers(packed, bn, stages, pg, wr, ar), pg,
+                      packed ? packed_stages(pg, bn, stages, wr, ar) : 0, wr);
 }
 
 // slabs per packed-weight copy for this problem and tile: 4 when K holds a whole number of
 // 4-slab runs and that plan fits in shared memory, else 1
-int packed_group(const Problem &p, int bn, int stages, int wr = kRowsW)
+int packed_group(const Problem &p, int bn, int stages, int wr = kRowsW, bool pair = false)
 {
     const int mode = mode_of(p.op);
     if (!(is_w4(mode) || mode == kW2A8)) return 1;
     const int kps = is_w4(mode) ? 64 : 128;
     if (p.K % kps || (p.K / kps) % 4) return 1;
-    return smem_bytes(mode, bn, stages, 4, wr) <= kMaxSmem ? 4 : 1;
+    return smem_bytes(mode, bn, stages, 4, wr, pair) <= kMaxSmem ? 4 : 1;
 }
 
-template <int MODE, int BN, int STAGES, int PG, bool TOKA = false>
+template <int MODE, int BN, int STAGES, int PG, bool TOKA = false, bool PAIR = false>
 cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
 {
     using T = Traits<MODE>;
-    using L = Smem<MODE, BN, STAGES, PG, TOKA>;
+    using L = Smem<MODE, BN, STAGES, PG, TOKA, PAIR>;
     if (L::total > kMaxSmem) return cudaErrorInvalidConfiguration;
-    auto kern = tc_gemm_kernel<MODE, BN, STAGES, PG, TOKA>;
+    auto kern = tc_gemm_kernel<MODE, BN, STAGES, PG, TOKA, PAIR>;
     // the dynamic shared-memory opt-in is per device: remember it per device
     static std::mutex mu;
     static bool opted_in[64] = {};
@@ -902,21 +1062,21 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.W, p.K, p.N, (uint64_t)p.K * 2, 64,
                       kRowsW, CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
-                      BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                      L::AR, CU_TENSOR_MAP_SWIZZLE_128B);
     } else if constexpr (MODE == kW8A8) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.W, p.K, p.N, (uint64_t)p.K, 128,
                       kRowsW, CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, L::AR,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     } else if constexpr (is_w4(MODE)) {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 8, p.N, (uint64_t)p.K / 2,
                       8 * PG, L::WR, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
              make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, p.A, p.K, p.M, (uint64_t)p.K * 2, 64,
-                      BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                      L::AR, CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
         ok = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.W, p.K / 16, p.N, (uint64_t)p.K / 4,
                       8 * PG, kRowsW, PG == 1 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B) &&
-             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, BN,
+             make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.A, p.K, p.M, (uint64_t)p.K, 128, L::AR,
                       CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (!ok) return cudaErrorInvalidValue;
@@ -924,29 +1084,54 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     const int nkb = (p.K + T::k_per_slab - 1) / T::k_per_slab;
     const int kbps = ((nkb + split_k - 1) / split_k + PG - 1) / PG * PG;   // whole copies
     const int splits = (nkb + kbps - 1) / kbps;
-    const int n_tiles = (p.N + L::WR - 1) / L::WR;
+    constexpr int UR = PAIR ? 2 * kRowsW : L::WR;      // weight rows per unit
+    const int n_tiles = (p.N + UR - 1) / UR;
     const int t_tiles = (p.M + BN - 1) / BN;
     const long units = (long)n_tiles * t_tiles * splits;
     if (units > 0x7fffffffL) return cudaErrorInvalidValue;
-    // persistent grid: as many CTAs as fit on the device at once (shared memory, threads and
-    // the TMEM columns each CTA holds), never more than there are units
-    static int per_sm[64] = {};
-    static int sm_count[64] = {};
-    if (!per_sm[dev]) {
-        int occ = 0, sms = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::total) !=
-                cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return cudaErrorInvalidConfiguration;
-        occ = std::min(occ, (int)(512 / tmem_cols<TOKA ? kRowsT : BN>()));
-        sm_count[dev] = sms;
-        per_sm[dev] = std::max(1, occ);
+    // persistent grid: as many CTAs (CTA pairs) as fit on the device at once (shared memory,
+    // threads and the TMEM columns each CTA holds), never more than there are units
+    static int per_dev[64] = {};
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = L::total;
+    cfg.stream = stream;
+    if constexpr (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
     }
-    const int grid = (int)std::min<long>(units, (long)per_sm[dev] * sm_count[dev]);
-    kern<<<grid, kThreads, L::total, stream>>>(
-        tw, ta, static_cast<const __half *>(p.scales),
+    if (!per_dev[dev]) {
+        int resident = 0;
+        if constexpr (PAIR) {
+            // clusters of two that fit at once (one CTA per SM: the kernel holds all of TMEM's
+            // columns at 256 tokens and most of shared memory)
+            cfg.gridDim = dim3(2);
+            if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess)
+                return cudaErrorInvalidConfiguration;
+        } else {
+            int occ = 0, sms = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, L::total) !=
+                    cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return cudaErrorInvalidConfiguration;
+            occ = std::min(occ, (int)(512 / tmem_cols<TOKA ? kRowsT : BN>()));
+            resident = std::max(1, occ) * sms;
+        }
+        if (resident <= 0) return cudaErrorInvalidConfiguration;
+        per_dev[dev] = resident;
+    }
+    const int slots = (int)std::min<long>(units, (long)per_dev[dev]);
+    cfg.gridDim = dim3(PAIR ? 2 * slots : slots);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, kern, tw, ta, static_cast<const __half *>(p.scales),
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, p.C, p.M, p.N, p.K, p.gs,
         kbps, (int)units, split_k > 1 ? 1 : 0, p.mult, err);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -996,10 +1181,31 @@ cudaError_t launch_toka(const Problem &p, const qgemm_config_t &c, unsigned int 
     }
 }
 
+// CTA pairs (bm = 256): weight-major tiles of 256 weight rows x BN tokens shared by two SMs
+// (grouped packed copies only)
+template <int MODE, int BN>
+cudaError_t launch_pair(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                        cudaStream_t stream)
+{
+    constexpr int PG = (is_w4(MODE) || is_w2(MODE)) ? 4 : 1;
+    switch (c.stages) {
+    case 3: return launch_t<MODE, BN, 3, PG, false, true>(p, c.split_k, err, stream);
+    case 4: return launch_t<MODE, BN, 4, PG, false, true>(p, c.split_k, err, stream);
+    case 5: return launch_t<MODE, BN, 5, PG, false, true>(p, c.split_k, err, stream);
+    case 8: return launch_t<MODE, BN, 8, PG, false, true>(p, c.split_k, err, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 template <int MODE>
 cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                       cudaStream_t stream)
 {
+    if (c.bm == 2 * kRowsW) {
+        if (c.bn == 128) return launch_pair<MODE, 128>(p, c, err, stream);
+        if (c.bn == 256) return launch_pair<MODE, 256>(p, c, err, stream);
+        return cudaErrorInvalidValue;
+    }
     switch (c.bn) {
     case 16: return launch_stages<MODE, 16>(p, c, err, stream);
     case 32: return launch_stages<MODE, 32>(p, c, err, stream);
@@ -1024,13 +1230,26 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
         return smem_bytes(kW4A16, kTokT, c.stages, pg, kRowsT) <= kMaxSmem &&
                dq_buffers(true, kTokT, c.stages, pg, kRowsT) >= 3;
     }
-    if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
-    if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 128 && c.stages == 8) ||
-          (c.bn <= 64 && c.stages == 16)))
-        return false;
     if (c.split_k < 1 || c.split_k > 64) return false;
-    if (smem_bytes(mode_of(p.op), c.bn, c.stages, packed_group(p, c.bn, c.stages)) > kMaxSmem)
-        return false;
+    if (c.bm == 2 * kRowsW) {
+        // CTA pair: 256 weight rows x 128 / 256 tokens, each CTA holding half of the tokens
+        const int mode = mode_of(p.op);
+        const bool packed = is_w4(mode) || mode == kW2A8;
+        if (c.bn != 128 && c.bn != 256) return false;
+        if (c.stages != 3 && c.stages != 4 && c.stages != 5 && c.stages != 8) return false;
+        if (packed && packed_group(p, c.bn, c.stages, kRowsW, true) != 4) return false;
+        if (smem_bytes(mode, c.bn, c.stages, packed ? 4 : 1, kRowsW, true) > kMaxSmem) return false;
+        if (packed && dq_buffers(true, c.bn, c.stages, 4, kRowsW, c.bn / 2) < want_dq(4, c.bn))
+            return false;
+    } else {
+        if (c.bm != 0 && c.bm != kRowsW) return false;
+        if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
+        if (!((c.stages >= 2 && c.stages <= 5) || (c.bn <= 128 && c.stages == 8) ||
+              (c.bn <= 64 && c.stages == 16)))
+            return false;
+        if (smem_bytes(mode_of(p.op), c.bn, c.stages, packed_group(p, c.bn, c.stages)) > kMaxSmem)
+            return false;
+    }
     if (p.op == QG_OP_W4A16 && (p.K % 32 || p.gs % 32 || p.K % p.gs)) return false;
     if (p.op == QG_OP_W2A8 && p.K % 64) return false;
     if (p.op == QG_OP_W8A8 && p.K % 16) return false;

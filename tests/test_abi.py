@@ -321,3 +321,23 @@ def test_half2_gemv_config_rules():
     for M, gs in ((9, 128), (1, 64), (1, 32)):
         with pytest.raises(qg.QGemmError):
             qg.qgemm_set_config(qg.OP_W4A16, M, 4096, 4096, gs, 1, ok)
+
+
+def test_pair_tile_rules():
+    """Tensor-core tiles shared by a CTA pair (bm = 256): 128 or 256 tokens, stages 3, 4, 5 or 8,
+    weight-major only; the library refuses other shapes of the config up front."""
+    ok = {"path": qg.PATH_TC, "rows": 0, "bm": 256, "bn": 256, "bk": 0, "stages": 4,
+          "split_k": 1, "swap_ab": 1}
+    for op, gs in ((qg.OP_W4A16, 128), (qg.OP_W8A8, -1), (qg.OP_W2A8, -1), (qg.OP_DENSE_F16, -1)):
+        packed = op in (qg.OP_W4A16, qg.OP_W2A8)
+        for bn, st in ((256, 3), (256, 4), (256, 5), (128, 8)) + (((256, 8),) if packed else ()):
+            cfg = {**ok, "bn": bn, "stages": st}
+            qg.qgemm_set_config(op, 512, 16384, 16384, gs, 0, cfg)
+            assert qg.qgemm_plan(op, 512, 16384, 16384, gs, 0)["bm"] == 256
+            qg.qgemm_set_config(op, 512, 16384, 16384, gs, 0, None)
+    for bad in ({"bn": 64}, {"stages": 2}, {"stages": 16}, {"bm": 192}, {"swap_ab": 0}):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, 512, 16384, 16384, 128, 1, {**ok, **bad})
+    # weights carried in the activation ring (fp16 / int8) leave no room for 8 stages of 256
+    with pytest.raises(qg.QGemmError):
+        qg.qgemm_set_config(qg.OP_DENSE_F16, 512, 16384, 16384, -1, 0, {**ok, "stages": 8})

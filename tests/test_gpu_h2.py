@@ -79,15 +79,20 @@ def test_h2_interleaved_layout():
 
 
 def test_h2_large_activations_inside_the_stated_range():
-    """|a| up to ~300 (runs of 16 centred products stay far from the fp16 limit)."""
-    M, N, K, gs = 1, 256, 4096, 128
+    """Activations scaled by 80 (|a| up to ~300): the fp16 runs stay finite and the result keeps
+    its relative accuracy. Products are rounded to fp16, so the absolute error grows with |A|:
+    the rule's absolute term is scaled by the same factor here (relative Frobenius unchanged)."""
+    M, N, K, gs, f = 1, 256, 4096, 128, 80.0
     case = W4Case(M, N, K, gs, 1, seed=3)
-    A = (case.h["A"].astype(np.float32) * 80.0).astype(np.float16)
+    A = (case.h["A"].astype(np.float32) * f).astype(np.float16)
     assert np.abs(A).max() < 512
     with pinned(qg.OP_W4A16, M, N, K, gs, 1, h2_cfg(64, 4, 1)):
         C = qg.qgemm_w4a16(to_dev(A), case.Wq, case.S, case.Z, group_size=gs)
+    got = C.float().cpu().numpy().astype(np.float64)
     ref = oracle.w4a16(A, case.Wq_host, case.h["scales"], case.h["zeros"], K, gs)
-    assert_fp16_close(C, ref, "large activations")
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - ref) <= f * oracle.ATOL + oracle.RTOL * np.abs(ref))
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) <= oracle.FROB
 
 
 def test_h2_split_overwrites_stale_output_and_keeps_guards():
