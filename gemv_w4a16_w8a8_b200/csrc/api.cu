@@ -302,6 +302,20 @@ qgemm_config_t heuristic(const Problem &p, int sms, bool allow_stream)
         if (tc_supports(p, tc)) return tc;
     }
     c.path = QG_PATH_GEMV;
+    if (p.op == QG_OP_W4A16 && p.M == 1 && p.gs % 128 == 0 && p.K % 128 == 0) {
+        // one token: the packed fp16 FMA-pipe GEMV (64-row tiles, 2-stage rings so that many
+        // CTAs fit per SM), K split until the tiles fill the SMs about six times over while every
+        // warp keeps at least four k-blocks
+        c.rows = 64;
+        c.bn = 2;
+        c.stages = 2;
+        const long tiles = (p.N + 63) / 64;
+        const long nkb = p.K / 128;
+        c.split_k = 1;
+        while (c.split_k < 16 && tiles * c.split_k < 6L * sms && nkb / (2L * c.split_k) >= 4)
+            c.split_k *= 2;
+        return c;
+    }
     if (p.op == QG_OP_W4A16) {
         c.rows = 32;
         const int kb = (p.gs % 128 == 0) ? 128 : (p.gs % 64 == 0 ? 64 : 32);
@@ -544,6 +558,20 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
             t.stages = st;
             if (tc_supports(p, t)) out.push_back(t);
         }
+    }
+    if ((p.op == QG_OP_DENSE_F16 || p.op == QG_OP_W8A8) && p.M >= 256) {
+        // the tile shared by a CTA pair (256 weight rows x 256 tokens): measured ahead of the
+        // single-CTA tile for fp16 / int8 weights only (the packed formats lose on the
+        // cross-SM hand-over of their upcast buffers)
+        qgemm_config_t t = tc_default(p, kDefaultSms);
+        t.bm = 256;
+        t.bn = 256;
+        for (int st : {4, 5})
+            for (int sk : {1, 2}) {
+                t.stages = st;
+                t.split_k = sk;
+                if (tc_supports(p, t)) out.push_back(t);
+            }
     }
     if (p.op == QG_OP_DENSE_F16 || p.M > 1) {
         const qgemm_config_t base = tc_default(p, kDefaultSms);
