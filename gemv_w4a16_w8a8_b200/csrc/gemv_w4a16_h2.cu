@@ -213,8 +213,11 @@ gemv_w4a16_h2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             }
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const float2 f = half2_bits_to_float2(run[t]);
-                acc[j][t] = fmaf(sc[j], fmaf(cz[j], asum[t], f.x + f.y), acc[j][t]);
+                // the run's two halves meet in fp16 (sums of 16 centred products each), then the
+                // group's scale and zero point apply in fp32
+                const uint32_t both = hadd2_u32(run[t], prmt(run[t], run[t], 0x1032));
+                const float f = __half2float(*reinterpret_cast<const __half *>(&both));
+                acc[j][t] = fmaf(sc[j], fmaf(cz[j], asum[t], f), acc[j][t]);
             }
         }
         consumed = i + 1;
