@@ -141,6 +141,24 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t
     return d;
 }
 
+// The same with the mask and the or-pattern as immediates (compile-time constants).
+template <uint32_t B, uint32_t C>
+__device__ __forceinline__ uint32_t lop3_and_or_i(uint32_t a)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(B), "n"(C));
+    return d;
+}
+
+// Byte permute with an immediate selector.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t prmt_i(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "n"(SEL));
+    return d;
+}
+
 // Byte permute: result byte i = byte sel_i of the 8-byte value {b:a}.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {

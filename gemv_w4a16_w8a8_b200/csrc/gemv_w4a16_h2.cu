@@ -60,10 +60,10 @@ __device__ __forceinline__ void centre_codes(uint32_t x, uint32_t (&w)[4])
     constexpr uint32_t kMagic = 0x64006400u, kLo = 0x000F000Fu, kHi = 0x00F000F0u;
     constexpr uint32_t k1032 = 0x64086408u, kInv16 = 0x2C002C00u, kNeg72 = 0xD480D480u;
     const uint32_t x8 = x >> 8;
-    w[0] = hsub2_u32(lop3_and_or(x, kLo, kMagic), k1032);
-    w[1] = hfma2_u32(lop3_and_or(x, kHi, kMagic), kInv16, kNeg72);
-    w[2] = hsub2_u32(lop3_and_or(x8, kLo, kMagic), k1032);
-    w[3] = hfma2_u32(lop3_and_or(x8, kHi, kMagic), kInv16, kNeg72);
+    w[0] = hsub2_u32(lop3_and_or_i<kLo, kMagic>(x), k1032);
+    w[1] = hfma2_u32(lop3_and_or_i<kHi, kMagic>(x), kInv16, kNeg72);
+    w[2] = hsub2_u32(lop3_and_or_i<kLo, kMagic>(x8), k1032);
+    w[3] = hfma2_u32(lop3_and_or_i<kHi, kMagic>(x8), kInv16, kNeg72);
 }
 
 // The activation pairs that meet centre_codes' output, word by word: natural packing pairs codes
@@ -77,10 +77,10 @@ __device__ __forceinline__ void act_pairs(const uint4 &v, uint32_t (&b)[4])
         b[2] = v.z;
         b[3] = v.w;
     } else {
-        b[0] = prmt(v.x, v.z, 0x5410);
-        b[1] = prmt(v.x, v.z, 0x7632);
-        b[2] = prmt(v.y, v.w, 0x5410);
-        b[3] = prmt(v.y, v.w, 0x7632);
+        b[0] = prmt_i<0x5410>(v.x, v.z);
+        b[1] = prmt_i<0x7632>(v.x, v.z);
+        b[2] = prmt_i<0x5410>(v.y, v.w);
+        b[3] = prmt_i<0x7632>(v.y, v.w);
     }
 }
 
@@ -173,7 +173,10 @@ gemv_w4a16_h2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             cz[j] = 8.f - half_bits_to_float(zbits[j]);
         }
         if (i + 1 < cnt) prefetch_sz(i + 1);
-        if (!mbar_wait(smem_u32(&full[warp][s]), (i / STAGES) & 1, abort_v, err)) break;
+        const uint32_t fbar = smem_u32(&full[warp][s]);
+        if (!(mbar_try_wait(fbar, (i / STAGES) & 1) ||
+              mbar_wait(fbar, (i / STAGES) & 1, abort_v, err)))
+            break;
         const uint8_t *slot = &ring[warp][s][0];
 
         // activations of this lane's 32 K values, paired like the codes; their sum in fp32
@@ -215,7 +218,7 @@ gemv_w4a16_h2_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_cons
             for (int t = 0; t < NT; ++t) {
                 // the run's two halves meet in fp16 (sums of 16 centred products each), then the
                 // group's scale and zero point apply in fp32
-                const uint32_t both = hadd2_u32(run[t], prmt(run[t], run[t], 0x1032));
+                const uint32_t both = hadd2_u32(run[t], prmt_i<0x1032>(run[t], run[t]));
                 const float f = __half2float(*reinterpret_cast<const __half *>(&both));
                 acc[j][t] = fmaf(sc[j], fmaf(cz[j], asum[t], f), acc[j][t]);
             }

@@ -298,10 +298,10 @@ __device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, 
     for (int j = 0; j < 4; ++j) {
         const uint32_t w = words[j], w8 = w >> 8;
         // natural packing: (q0,q4) (q1,q5) (q2,q6) (q3,q7); interleaved: (q0,q1) .. (q6,q7)
-        const uint32_t h0 = hsub2_u32(lop3_and_or(w, kLo, kMagic), kMagic);
-        const uint32_t h1 = hfma2_u32(lop3_and_or(w, kHi, kMagic), kInv16, kNeg64);
-        const uint32_t h2 = hsub2_u32(lop3_and_or(w8, kLo, kMagic), kMagic);
-        const uint32_t h3 = hfma2_u32(lop3_and_or(w8, kHi, kMagic), kInv16, kNeg64);
+        const uint32_t h0 = hsub2_u32(lop3_and_or_i<kLo, kMagic>(w), kMagic);
+        const uint32_t h1 = hfma2_u32(lop3_and_or_i<kHi, kMagic>(w), kInv16, kNeg64);
+        const uint32_t h2 = hsub2_u32(lop3_and_or_i<kLo, kMagic>(w8), kMagic);
+        const uint32_t h3 = hfma2_u32(lop3_and_or_i<kHi, kMagic>(w8), kInv16, kNeg64);
         uint4 o;
         if constexpr (ILV) {
             o.x = hfma2_u32(h0, sc, nz);
@@ -309,10 +309,10 @@ __device__ __forceinline__ void dequant_w4(const uint4 &p, uint8_t *dst, int r, 
             o.z = hfma2_u32(h2, sc, nz);
             o.w = hfma2_u32(h3, sc, nz);
         } else {
-            o.x = hfma2_u32(prmt(h0, h1, 0x5410), sc, nz);   // (q0, q1)
-            o.y = hfma2_u32(prmt(h2, h3, 0x5410), sc, nz);   // (q2, q3)
-            o.z = hfma2_u32(prmt(h0, h1, 0x7632), sc, nz);   // (q4, q5)
-            o.w = hfma2_u32(prmt(h2, h3, 0x7632), sc, nz);   // (q6, q7)
+            o.x = hfma2_u32(prmt_i<0x5410>(h0, h1), sc, nz);   // (q0, q1)
+            o.y = hfma2_u32(prmt_i<0x5410>(h2, h3), sc, nz);   // (q2, q3)
+            o.z = hfma2_u32(prmt_i<0x7632>(h0, h1), sc, nz);   // (q4, q5)
+            o.w = hfma2_u32(prmt_i<0x7632>(h2, h3), sc, nz);   // (q6, q7)
         }
         *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }
@@ -342,10 +342,10 @@ __device__ __forceinline__ void dequant_w2(const uint4 &p, uint8_t *dst, int r, 
         if constexpr (ILV) {
             o = make_uint4(d0, d1, d2, d3);
         } else {
-            o.x = prmt(d0, d1, 0x5140);   // values 0, 1, 2, 3
-            o.y = prmt(d0, d1, 0x7362);   // 4 .. 7
-            o.z = prmt(d2, d3, 0x5140);   // 8 .. 11
-            o.w = prmt(d2, d3, 0x7362);   // 12 .. 15
+            o.x = prmt_i<0x5140>(d0, d1);   // values 0, 1, 2, 3
+            o.y = prmt_i<0x7362>(d0, d1);   // 4 .. 7
+            o.z = prmt_i<0x5140>(d2, d3);   // 8 .. 11
+            o.w = prmt_i<0x7362>(d2, d3);   // 12 .. 15
         }
         *reinterpret_cast<uint4 *>(row + (((4 * h + j) ^ (r & 7)) << 4)) = o;
     }

@@ -88,9 +88,15 @@ typedef enum qg_path {
 typedef struct qgemm_config_t {
     int32_t path;    /* qg_path                                                             */
     int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise)  */
-    int32_t bm;      /* TC: tile extent along the MMA's M (128)                              */
-    int32_t bn;      /* TC: tile extent along the MMA's N. GEMV (W4A16, stages > 0, M = 1):
-                        1 = products on the FMA pipe instead of the warp-level MMA           */
+    int32_t bm;      /* TC: tile extent along the MMA's M: 128 (one CTA), or 256 for the
+                        weight-major tile shared by a CTA pair (one cta_group::2 MMA over
+                        two SMs: 256 weight rows, bn = 128 or 256 tokens, stages 3, 4, 5 or 8) */
+    int32_t bn;      /* TC: tile extent along the MMA's N. GEMV (W4A16, stages > 0):
+                        1 = one token, exact fp16 products summed in fp32 on the FMA pipe;
+                        2 = 1..8 tokens on the packed fp16 FMA pipe (rows 32 or 64 per CTA,
+                        stages 2..6, group size a multiple of 128): products of the centred
+                        codes summed in fp16 over 16 per lane and K run of 32, fp32 across
+                        runs, so the absolute error grows with |A| (keep |A| < 512)        */
     int32_t bk;      /* TC: tile extent along K                                              */
     int32_t stages;  /* TC: activation ring depth (2..5; 8 for bn <= 128, 16 for bn <= 64;
                         2..4 when swap_ab = 0)                                               */
