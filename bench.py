@@ -20,8 +20,9 @@ The headline workload (--workload, default the N = K = 16384 W4A16 sweep over M)
 Unless --no-extras, the other benchmark configurations are timed after it, shape by shape, into
 "configs" of the same line: one-token W4A16 at K = N = 4096 with split_k 1 and 4, the LLaMA-style
 shapes with and without zero points, W8A8 and W2A8 over M at N = K = 16384, W4A16 without zero
-points and the dense fp16 baseline at M = 512 / 16384, and a sweep of the tensor-core pipeline
-depth (stages 2..5) on the large-M shapes.
+points and the dense fp16 baseline at M = 512 / 16384, the same W4A16 codes in the pre-shuffled
+(interleaved) int4 layout, and a sweep of the tensor-core pipeline depth (stages 2..5) on the
+large-M shapes.
 
 Prints one JSON line (rank 0). Under torchrun every rank runs the same workload on its own GPU
 (independent replicas, no collective on the data path); `value` is the whole-job throughput
@@ -81,6 +82,10 @@ WORKLOADS = {
     # the compute-bound shapes: W4A16 without zero points, and the dense fp16 baseline
     "w4a16_nozero_large_m": {"op": "w4a16", "has_zero": 0,
                              "shapes": [(512, 16384, 16384), (16384, 16384, 16384)]},
+    # the same codes in the pre-shuffled (interleaved) int4 layout, zero points as the headline
+    "w4a16_interleaved": {"op": "w4a16", "has_zero": 1, "layout": "interleaved",
+                          "shapes": [(1, 16384, 16384), (128, 16384, 16384), (512, 16384, 16384),
+                                     (16384, 16384, 16384)]},
     "dense_large_m": {"op": "dense", "has_zero": 0,
                       "shapes": [(512, 16384, 16384), (16384, 16384, 16384)]},
 }
@@ -104,18 +109,19 @@ EXTRAS = [
     ("w8a8_nk16384", "w8a8_nk16384", (1, 4), False),
     ("w2a8_nk16384", "w2a8_nk16384", (), False),
     ("w4a16_nozero_large_m", "w4a16_nozero_large_m", (), True),
+    ("w4a16_interleaved", "w4a16_interleaved", (), False),
     ("dense_large_m", "dense_large_m", (), True),
 ]
 SWEEP_STAGES = (2, 3, 4, 5)
 
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum):
-# the weight-major tile (256 tokens, 3 stages) on M = 2048, N = K = 16384 measured 605.2 MB read
-# + 60.9 MB written; an M = 16384 launch runs the same pattern (8 token tiles against all 128
-# weight tiles, weights read once per group) 8 times, so its traffic is scaled by 8.
-TRAFFIC_BYTES = {(16384, 16384, 16384): 8 * (605178368 + 60862208)}
-TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 2048 launch of the "
-                  "same tile, scaled by its 8 groups of token tiles")
+# the weight-major tile (256 tokens, 3 stages) on M = 4096, N = K = 16384 measured 1271.105 MB read
+# + 129.454 MB written; an M = 16384 launch runs the same pattern (groups of 8 token tiles against
+# all 128 weight tiles, weights read once per group) 4 times as often, so its traffic is scaled by 4.
+TRAFFIC_BYTES = {(16384, 16384, 16384): 4 * (1271105000 + 129453568)}
+TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 4096 launch of the "
+                  "same tile, scaled by 4 (its 2 groups of 8 token tiles against 8)")
 
 
 def shape_bytes(op, M, K, N, has_zero, gs=GS):
@@ -321,8 +327,10 @@ def merge_parity(items):
 
 # ---- our arm ----------------------------------------------------------------------------------------
 
-def op_code(op):
+def op_code(op, sp=None):
     import gemv_w4a16_w8a8_b200 as qg
+    if op == "w4a16" and sp is not None and sp.get("ilv"):
+        return qg.OP_W4A16_INTERLEAVED
     return {"w4a16": qg.OP_W4A16, "w8a8": qg.OP_W8A8, "w2a8": qg.OP_W2A8,
             "dense": qg.OP_DENSE_F16}[op]
 
@@ -338,17 +346,17 @@ def host_inputs(op, M, K, N, hz, seed):
     return synth.dense_inputs(M, N, K, seed=seed)
 
 
-def prepare_shape(op, M, K, N, hz, seed, dev, pinned=True):
+def prepare_shape(op, M, K, N, hz, seed, dev, pinned=True, ilv=False):
     """Seeded inputs of one shape in HBM (weights replicated into enough copies, >= 3x L2 in
     total, that consecutive calls never find theirs in L2), plus page-locked host copies of A
     and C for the end-to-end form. The host arrays stay in sp["h"] for the parity leg."""
     import torch
     import gemv_w4a16_w8a8_b200 as qg
     h = host_inputs(op, M, K, N, hz, seed)
-    sp = {"M": M, "K": K, "N": N, "hz": hz, "seed": seed, "h": h}
+    sp = {"M": M, "K": K, "N": N, "hz": hz, "seed": seed, "h": h, "ilv": ilv}
     if op == "w4a16":
         codes = torch.from_numpy(h["codes"]).to(dev)
-        W0 = qg.quant_pack_int4(codes)
+        W0 = (qg.quant_pack_int4_interleaved if ilv else qg.quant_pack_int4)(codes)
         del codes
         sp["S"] = torch.from_numpy(h["scales"]).to(dev)
         sp["Z"] = torch.from_numpy(h["zeros"]).to(dev) if hz else None
@@ -378,7 +386,8 @@ def matmul(op, sp, W, split_k=0, A=None, C=None):
     A = sp["A"] if A is None else A
     C = sp["C"] if C is None else C
     if op == "w4a16":
-        qg.qgemm_w4a16(A, W, sp["S"], sp["Z"], C=C, group_size=GS, split_k=split_k)
+        mm = qg.qgemm_w4a16_interleaved if sp.get("ilv") else qg.qgemm_w4a16
+        mm(A, W, sp["S"], sp["Z"], C=C, group_size=GS, split_k=split_k)
     elif op == "w8a8":
         qg.qgemm_w8a8(A, W, C=C, split_k=split_k)
     elif op == "w2a8":
@@ -392,8 +401,8 @@ def tune_shape(op, sp, hz, no_tune, reps):
     M, K, N = sp["M"], sp["K"], sp["N"]
     g_op = GS if op == "w4a16" else -1
     if no_tune:
-        return qg.qgemm_plan(op_code(op), M, N, K, g_op, hz)
-    return qg.qgemm_tune(op_code(op), sp["A"], sp["W"][0], sp.get("S"), sp.get("Z"), sp["C"],
+        return qg.qgemm_plan(op_code(op, sp), M, N, K, g_op, hz)
+    return qg.qgemm_tune(op_code(op, sp), sp["A"], sp["W"][0], sp.get("S"), sp.get("Z"), sp["C"],
                          M, N, K, g_op, hz, reps=reps)
 
 
@@ -445,12 +454,13 @@ def run_extras(args, dev, peaks, headline_sps, deadline):
             continue
         wl = WORKLOADS[wl_name]
         op, hz = wl["op"], wl["has_zero"]
+        ilv = wl.get("layout") == "interleaved"
         rows = []
         for si, (M, K, N) in enumerate(wl["shapes"]):
-            sp = prepare_shape(op, M, K, N, hz, 7000 + 100 * si + hz, dev, pinned=False)
+            sp = prepare_shape(op, M, K, N, hz, 7000 + 100 * si + hz, dev, pinned=False, ilv=ilv)
             g_op = GS if op == "w4a16" else -1
             for s in splits:   # the planner's path at the stated split, before the search
-                cfg = qg.qgemm_plan(op_code(op), M, N, K, g_op, hz, s)
+                cfg = qg.qgemm_plan(op_code(op, sp), M, N, K, g_op, hz, s)
                 ms = time_shape(op, sp, split_k=s)
                 par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"])
                 rows.append(shape_row(op, sp, ms, cfg, peaks, par, split_req=s))
@@ -464,6 +474,8 @@ def run_extras(args, dev, peaks, headline_sps, deadline):
             del sp
             torch.cuda.empty_cache()
         out[name] = {"op": op, "has_zero": hz, "per_shape": rows}
+        if ilv:
+            out[name]["layout"] = "interleaved"
     # the headline's own large-M W4A16 shapes (zero points) in the stage sweep
     for sp in headline_sps:
         if sp["M"] >= 512 and time.time() <= deadline:
@@ -484,7 +496,7 @@ def stage_sweep(op, sp, tuned, peaks):
         cfg = dict(tuned)
         cfg["stages"] = st
         try:
-            qg.qgemm_set_config(op_code(op), M, N, K, g_op, hz, cfg)
+            qg.qgemm_set_config(op_code(op, sp), M, N, K, g_op, hz, cfg)
         except qg.QGemmError:
             rows.append({"op": op, "shape_mkn": [M, K, N], "has_zero": hz, "stages": st,
                          "cfg": cfg, "us": None, "note": "does not fit shared memory"})
@@ -494,7 +506,7 @@ def stage_sweep(op, sp, tuned, peaks):
         r = shape_row(op, sp, ms, cfg, peaks, par)
         r.update({"op": op, "stages": st})
         rows.append(r)
-    qg.qgemm_set_config(op_code(op), M, N, K, g_op, hz, tuned)
+    qg.qgemm_set_config(op_code(op, sp), M, N, K, g_op, hz, tuned)
     return rows
 
 
