@@ -735,7 +735,8 @@ def run_e2e(args, op, per_shape, hz, stream, world, dev, flops_step):
     h2d = sum(sp["A_host"].numel() * sp["A_host"].element_size() for sp in per_shape)
     d2h = sum(sp["C_host"].numel() * sp["C_host"].element_size() for sp in per_shape)
     if op == "w4a16":
-        ws_bytes = max(qg.qgemm_w4a16_host_workspace_bytes(sp["M"], sp["N"], sp["K"], 0)
+        ws_bytes = max(qg.qgemm_w4a16_host_workspace_bytes(sp["M"], sp["N"], sp["K"],
+                                                           args.e2e_chunk)
                        for sp in per_shape)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
@@ -765,8 +766,9 @@ def run_e2e(args, op, per_shape, hz, stream, world, dev, flops_step):
     # the host-side results of the last step, sampled against the oracle
     par = merge_parity([parity_check(op, sp["h"], sp["C_host"], sp["M"], sp["K"], sp["N"], hz,
                                      sp["seed"] + 1) for sp in per_shape])
-    path = ("qgemm_w4a16_host (pinned host A and C, chunks of up to 2048 tokens, copies in both "
-            "directions overlapped with the matmul)" if op == "w4a16" else
+    path = (f"qgemm_w4a16_host (pinned host A and C, chunks of up to "
+            f"{args.e2e_chunk or 1024} tokens, copies in both directions overlapped with the "
+            f"matmul)" if op == "w4a16" else
             "pinned host A copied in, the call, C copied out, on one stream")
     return {"value": round(value, 3), "unit": UNITS[op],
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
@@ -902,6 +904,8 @@ def main(argv=None):
                     help="time only the headline workload")
     ap.add_argument("--extras-budget", type=float, default=240.0,
                     help="seconds after which the remaining extra configurations are skipped")
+    ap.add_argument("--e2e-chunk", type=int, default=0,
+                    help="tokens per chunk of the host-buffer form (0: the library's default)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
     args = ap.parse_args(argv)

@@ -711,7 +711,7 @@ qg_status qgemm_w4a16_splitk_f32(const void *A, const uint32_t *Wq, const void *
 size_t qgemm_w4a16_host_workspace_bytes(int M, int N, int K, int chunk_tokens)
 {
     if (M <= 0 || N <= 0 || K <= 0 || chunk_tokens < 0) return 0;
-    const size_t mc = chunk_tokens ? (size_t)std::min(chunk_tokens, M) : (size_t)std::min(M, 2048);
+    const size_t mc = chunk_tokens ? (size_t)std::min(chunk_tokens, M) : (size_t)std::min(M, 1024);
     const size_t a = (mc * K * 2 + 255) / 256 * 256, c = (mc * N * 2 + 255) / 256 * 256;
     return 2 * (a + c);
 }

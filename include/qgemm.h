@@ -208,7 +208,7 @@ qg_status qgemm_w4a16_host(const void *A_host, const uint32_t *Wq, const void *s
                            int split_k, int has_zero, void *workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
-/* Workspace bytes for qgemm_w4a16_host with chunks of chunk_tokens tokens (0: min(M, 2048));
+/* Workspace bytes for qgemm_w4a16_host with chunks of chunk_tokens tokens (0: min(M, 1024));
  * 0 if the arguments are invalid. */
 size_t qgemm_w4a16_host_workspace_bytes(int M, int N, int K, int chunk_tokens);
 
