@@ -115,13 +115,15 @@ EXTRAS = [
 SWEEP_STAGES = (2, 3, 4, 5)
 
 
-# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum):
-# the weight-major tile (256 tokens, 3 stages) on M = 4096, N = K = 16384 measured 1271.105 MB read
-# + 129.454 MB written; an M = 16384 launch runs the same pattern (groups of 8 token tiles against
-# all 128 weight tiles, weights read once per group) 4 times as often, so its traffic is scaled by 4.
-TRAFFIC_BYTES = {(16384, 16384, 16384): 4 * (1271105000 + 129453568)}
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum),
+# by weight-major token tile: on M = 4096, N = K = 16384 the 256-token tile (3 stages) read
+# 1271.105 MB and wrote 129.454 MB; the 512-token tile (4 half-tile stages) read 816.418 MB and
+# wrote 120.399 MB. An M = 16384 launch runs the same pattern (groups of 2048 tokens against all
+# 128 weight tiles, weights read once per group) 4 times as often, so its traffic is scaled by 4.
+TRAFFIC_BYTES = {(16384, 16384, 16384, 256): 4 * (1271105000 + 129453568),
+                 (16384, 16384, 16384, 512): 4 * (816417536 + 120399104)}
 TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 4096 launch of the "
-                  "same tile, scaled by 4 (its 2 groups of 8 token tiles against 8)")
+                  "same tile, scaled by 4 (its 2 groups of 2048 tokens against 8)")
 
 
 def shape_bytes(op, M, K, N, has_zero, gs=GS):
@@ -640,9 +642,9 @@ def run_ours(args, world, rank, local):
     roof = roofline_of(op, M, K, N, hz, shape_ms[j], peaks, burst=timed_alone)
     if args.traffic is not None:
         roof["traffic"] = args.traffic
-    elif (M, K, N) in TRAFFIC_BYTES and sp["cfg"]["path"] == 2 and sp["cfg"]["bn"] == 256 and \
-            sp["cfg"]["swap_ab"] == 1:
-        roof["traffic"] = TRAFFIC_BYTES[(M, K, N)]
+    elif (M, K, N, sp["cfg"]["bn"]) in TRAFFIC_BYTES and sp["cfg"]["path"] == 2 and \
+            sp["cfg"]["swap_ab"] == 1 and sp["cfg"]["bm"] in (0, 128) and sp["cfg"]["rows"] == 0:
+        roof["traffic"] = TRAFFIC_BYTES[(M, K, N, sp["cfg"]["bn"])]
         roof["traffic_source"] = TRAFFIC_SOURCE
     else:
         roof["traffic"] = None

@@ -222,6 +222,10 @@ constexpr int kSinkBytes = 256 * 4;
 constexpr int min_dq(int pg, int bn) { return (pg < 2 || per_slab_handoff(bn)) ? 2 : pg; }
 constexpr int want_dq(int pg, int bn) { return per_slab_handoff(bn) ? 3 : min_dq(pg, bn); }
 
+// Activation rows of one stage held by a CTA: the token tile; half of it for a CTA pair; 256 for
+// the 512-token tile, whose slabs arrive as two 256-token stages (one per accumulator).
+constexpr int act_rows(int bn, bool pair) { return pair ? bn / 2 : (bn > 256 ? 256 : bn); }
+
 // ar: activation rows of a stage held by this CTA (the MMA's N, or half of it for a CTA pair)
 constexpr int smem_total(bool packed, int ar, int stages, int dq, int pg, int sp, int wr = kRowsW)
 {
@@ -263,7 +267,7 @@ constexpr int dq_buffers(bool packed, int bn, int stages, int pg, int wr = kRows
 template <int MODE, int BN, int STAGES, int PG, bool TOKA = false, bool PAIR = false> struct Smem {
     static constexpr bool packed = Traits<MODE>::packed;
     static constexpr int WR = wrows<TOKA>();
-    static constexpr int AR = PAIR ? BN / 2 : BN;
+    static constexpr int AR = act_rows(BN, PAIR);
     static constexpr int a_bytes = AR * kSlabBytes;
     static constexpr int w_bytes = kRowsW * kSlabBytes;          // dense / int8 weight slab
     static constexpr int pw_bytes = WR * 32 * PG;                // packed weight copy (PG slabs)
@@ -363,15 +367,15 @@ struct Unit {
 };
 
 __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv, int nkb,
-                                        int kbps, int wr = kRowsW)
+                                        int kbps, int wr = kRowsW, int group_t = kGroupT)
 {
     const int tiles = n_tiles * t_tiles;
     const int split = u / tiles;
     const int tile = u - split * tiles;
-    const int per_group = kGroupT * n_tiles;
+    const int per_group = group_t * n_tiles;
     const int group = tile / per_group;
-    const int first_t = group * kGroupT;
-    const int gt = min(kGroupT, t_tiles - first_t);
+    const int first_t = group * group_t;
+    const int gt = min(group_t, t_tiles - first_t);
     const int within = tile - group * per_group;
     Unit w;
     w.t0 = (first_t + within % gt) * BNv;
@@ -403,8 +407,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     static_assert(!TOKA || (is_w4(MODE) && BN == kTokT), "token-major tiles: W4A16, 128 tokens");
     static_assert(!PAIR || (!TOKA && BN >= 128), "CTA pairs: weight-major tiles of 128+ tokens");
     constexpr int WR = L::WR;
-    constexpr int NMMA = TOKA ? kRowsT : BN;          // the MMA's N (accumulator columns)
-    constexpr uint32_t kCols = tmem_cols<NMMA>();
+    // DUAL (BN = 512, packed weights): each upcast weight slab feeds two MMAs, one per 256-token
+    // half of the tile, into two accumulators that fill TMEM (no double buffering); the halves
+    // arrive as consecutive activation stages
+    constexpr bool DUAL = BN == 512;
+    static_assert(!DUAL || (L::packed && !TOKA && !PAIR && STAGES % 2 == 0),
+                  "512-token tiles: packed weights, weight-major, single CTA, even stages");
+    constexpr int NH = DUAL ? 2 : 1;                  // activation stages per slab
+    constexpr int BH = BN / NH;                       // tokens per activation stage
+    constexpr int NMMA = TOKA ? kRowsT : BH;          // the MMA's N (accumulator columns)
+    constexpr uint32_t kCols = DUAL ? 512u : tmem_cols<NMMA>();
+    constexpr int NBUF = DUAL ? 1 : 2;                // accumulator buffers in TMEM
+    constexpr int GT = DUAL ? kGroupT / 2 : kGroupT;  // token tiles per raster group
     constexpr uint32_t kIdesc = instr_desc<MODE, NMMA, PAIR ? 2 * kRowsW : kRowsW>();
     // CTA pairs: a unit covers UR = 256 weight rows, this CTA's 128 start at roff, and this CTA
     // loads tokens aoff .. aoff + AR - 1 of the tile; both CTAs walk the same units
@@ -506,14 +520,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         int it = 0;
         bool stop = false;
         for (int u = ustart; u < units && !stop; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
-            for (int i = 0; i < w.nk; ++i, ++it) {
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+            for (int i = 0; i < NH * w.nk; ++i, ++it) {
                 const int s = it % STAGES;
                 if (!warp_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
                     stop = true;
                     break;
                 }
-                const int kx = (w.kb0 + i) * T::k_per_slab;
+                // stage it holds K slab i / NH of tokens t0 + (i % NH) * BH .. + BH - 1
+                const int kx = (w.kb0 + i / NH) * T::k_per_slab;
+                const int ty = w.t0 + (i % NH) * BH;
                 if (lane == 0) {
                     if constexpr (PAIR) {
                         // both CTAs' copies complete on the leader's barrier, which expects both
@@ -522,11 +538,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                         if constexpr (!L::packed)
                             tma_load_2d_pair(smem_u32(w_tma(s)), &tm_w, fb, kx, w.n0 + roff);
                         tma_load_2d_pair(smem_u32(a_tile(s)), &tm_a, fb, kx, w.t0 + aoff);
+                    } else if (DUAL && ty >= M) {
+                        // a half with no tokens: no copy; its accumulator columns are never stored
+                        mbar_arrive(full_bar(s));
                     } else {
                         mbar_expect_tx(full_bar(s), kTx);
                         if constexpr (!L::packed)
                             tma_load_2d(smem_u32(w_tma(s)), &tm_w, full_bar(s), kx, w.n0);
-                        tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kx, w.t0);
+                        tma_load_2d(smem_u32(a_tile(s)), &tm_a, full_bar(s), kx, ty);
                     }
                 }
                 __syncwarp();
@@ -551,7 +570,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             int it = 0;
             bool stop = false;
             for (int u = ustart; u < units && !stop; u += ustep) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
                 // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
                 for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
@@ -575,30 +594,54 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     } else if (warp == 5 && (!PAIR || rank == 0)) {
         // ---------------- MMA issuer (a pair's leader issues for both CTAs) ----------------
         // Lane 0 issues the MMAs and the commits: a commit tracks the MMAs its own thread issued.
-        int it = 0, j = 0;
+        int it = 0, sa = 0, j = 0;   // slabs, activation stages and units consumed
         bool stop = false;
         for (int u = ustart; u < units && !stop; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
             if (w.nk == 0) continue;
-            const int b = j & 1;
-            if (!warp_wait(acce_bar(b), ((j >> 1) & 1) ^ 1, abort_flag, err)) break;
+            const int b = NBUF == 2 ? j & 1 : 0;
+            const int use = NBUF == 2 ? j >> 1 : j;     // earlier uses of buffer b
+            if (!warp_wait(acce_bar(b), (use & 1) ^ 1, abort_flag, err)) break;
             tc_fence_after();
             const uint32_t dtm = tmem_base + (uint32_t)(b * NMMA);
             // one slab at a time: wait for its activation stage (and upcast weights), issue its 4
             // MMAs, then commit its buffers back at once, so that every buffer returns to its
             // producer as soon as the tensor core is done with it (a commit tracks all MMAs this
             // thread issued before it)
-            for (int i = 0; i < w.nk; ++i, ++it) {
-                const int s = it % STAGES;
+            for (int i = 0; i < w.nk; ++i, ++it, sa += NH) {
+                const int s = sa % STAGES;
                 const int d = T::packed ? it % DQ : 0;
                 bool ready = true;
                 if constexpr (T::packed) ready = warp_wait(dqf_bar(d), (it / DQ) & 1, abort_flag, err);
-                ready = ready && warp_wait(full_bar(s), (it / STAGES) & 1, abort_flag, err);
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    ready = ready && warp_wait(full_bar((sa + h) % STAGES), ((sa + h) / STAGES) & 1,
+                                               abort_flag, err);
                 if (!ready) {
                     stop = true;
                     break;
                 }
                 tc_fence_after();
+                if constexpr (DUAL) {
+                    // the upcast slab against both 256-token halves: 4 MMAs into each accumulator,
+                    // each half's activation stage released once its MMAs are done
+                    const uint64_t wdesc = sw128_desc(smem_u32(w_dq(d)));
+                    if (lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
+                            const int sh = (sa + h) % STAGES;
+                            const uint64_t tdesc = sw128_desc(smem_u32(a_tile(sh)));
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                mma_issue<MODE>(dtm + (uint32_t)(h * BH), wdesc + 2 * k, tdesc + 2 * k,
+                                                kIdesc, (i | k) != 0 ? 1u : 0u);
+                            mma_commit(empty_bar(sh));
+                        }
+                        mma_commit(dqe_bar(d));
+                    }
+                    __syncwarp();
+                    continue;
+                }
                 const uint64_t wdesc = sw128_desc(smem_u32(T::packed ? w_dq(d) : w_tma(s)));
                 const uint64_t tdesc = sw128_desc(smem_u32(a_tile(s)));
                 const uint64_t adesc = TOKA ? tdesc : wdesc, bdesc = TOKA ? wdesc : tdesc;
@@ -660,10 +703,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 while (c.u < units && c.i >= c.w.nk) {
                     c.u += ustep;
                     c.i = 0;
-                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
                 }
             };
-            Cursor cur{ustart, 0, unit_of(ustart, n_tiles, t_tiles, BN, nkb, kb_per_split, UR)};
+            Cursor cur{ustart, 0, unit_of(ustart, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT)};
             settle(cur);
             // Scales and zeros. Per slab a thread needs s[n][g] and z[n][g] of its row n. Loading
             // those 2-byte values one slab at a time makes every warp touch 32 rows (32 sectors)
@@ -695,7 +738,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             };
             // the window after wnd in this CTA's walk (same unit, or the next unit's first one)
             auto next_window = [&](Window &out, const Window &wnd) {
-                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
                 const int g_last = min(((w.kb0 + w.nk) * 64 - 1) / gs, G - 1);
                 if (wnd.gb + 8 <= g_last) {
                     load_window(out, wnd.u, w, wnd.gb + 8);
@@ -704,7 +747,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 int u = wnd.u + ustep;
                 Unit nw = w;
                 while (u < units) {
-                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
                     if (nw.nk > 0) break;
                     u += ustep;
                 }
@@ -883,10 +926,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         const bool pairs = (N & 1) == 0;
         int j = 0;
         for (int u = ustart; u < units; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
             if (w.nk == 0) continue;
-            const int b = j & 1;
-            bool ok = mbar_wait(accf_bar(b), (j >> 1) & 1, abort_flag, err);
+            const int b = NBUF == 2 ? j & 1 : 0;
+            bool ok = mbar_wait(accf_bar(b), (NBUF == 2 ? j >> 1 : j) & 1, abort_flag, err);
             tc_fence_after();
             // tcgen05.ld is warp-collective: decide per warp, never per lane
             ok = __all_sync(0xffffffffu, ok && !*abort_flag);
@@ -1018,7 +1061,7 @@ int mode_of(int op)
 int smem_bytes(int mode, int bn, int stages, int pg, int wr = kRowsW, bool pair = false)
 {
     const bool packed = (is_w4(mode) || mode == kW2A8);
-    const int ar = pair ? bn / 2 : bn;
+    const int ar = act_rows(bn, pair);
     return smem_total(packed, ar, stages, dq_buffers(packed, bn, stages, pg, wr, ar), pg,
                       packed ? packed_stages(pg, bn, stages, wr, ar) : 0, wr);
 }
@@ -1119,7 +1162,7 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
                     cudaSuccess ||
                 cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
                 return cudaErrorInvalidConfiguration;
-            occ = std::min(occ, (int)(512 / tmem_cols<TOKA ? kRowsT : BN>()));
+            occ = std::min(occ, BN > 256 ? 1 : (int)(512 / tmem_cols<TOKA ? kRowsT : BN>()));
             resident = std::max(1, occ) * sms;
         }
         if (resident <= 0) return cudaErrorInvalidConfiguration;
@@ -1197,6 +1240,25 @@ cudaError_t launch_pair(const Problem &p, const qgemm_config_t &c, unsigned int 
     }
 }
 
+// 512-token weight-major tiles (packed weights): two 256-token accumulators fed by each upcast
+// slab, activation stages in pairs
+template <int MODE>
+cudaError_t launch_dual(const Problem &p, const qgemm_config_t &c, unsigned int *err,
+                        cudaStream_t stream)
+{
+    if constexpr (is_w4(MODE) || is_w2(MODE)) {
+        const bool g4 = packed_group(p, 512, c.stages) == 4;
+        switch (c.stages) {
+        case 2: return g4 ? launch_t<MODE, 512, 2, 4>(p, c.split_k, err, stream)
+                          : launch_t<MODE, 512, 2, 1>(p, c.split_k, err, stream);
+        case 4: return g4 ? launch_t<MODE, 512, 4, 4>(p, c.split_k, err, stream)
+                          : launch_t<MODE, 512, 4, 1>(p, c.split_k, err, stream);
+        default: break;
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
 template <int MODE>
 cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *err,
                       cudaStream_t stream)
@@ -1212,6 +1274,7 @@ cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *e
     case 64: return launch_stages<MODE, 64>(p, c, err, stream);
     case 128: return launch_stages<MODE, 128>(p, c, err, stream);
     case 256: return launch_stages<MODE, 256>(p, c, err, stream);
+    case 512: return launch_dual<MODE>(p, c, err, stream);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -1241,6 +1304,15 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
         if (smem_bytes(mode, c.bn, c.stages, packed ? 4 : 1, kRowsW, true) > kMaxSmem) return false;
         if (packed && dq_buffers(true, c.bn, c.stages, 4, kRowsW, c.bn / 2) < want_dq(4, c.bn))
             return false;
+    } else if (c.bn == 512) {
+        // two 256-token accumulators per upcast slab: packed weights, activation stages in pairs
+        const int mode = mode_of(p.op);
+        if (!(is_w4(mode) || mode == kW2A8)) return false;
+        if (c.bm != 0 && c.bm != kRowsW) return false;
+        if (c.stages != 2 && c.stages != 4) return false;
+        const int pg = packed_group(p, 512, c.stages);
+        if (smem_bytes(mode, 512, c.stages, pg) > kMaxSmem) return false;
+        if (dq_buffers(true, 512, c.stages, pg, kRowsW, 256) < want_dq(pg, 512)) return false;
     } else {
         if (c.bm != 0 && c.bm != kRowsW) return false;
         if (c.bn != 16 && c.bn != 32 && c.bn != 64 && c.bn != 128 && c.bn != 256) return false;
@@ -1260,7 +1332,8 @@ bool tc_supports(const Problem &p, const qgemm_config_t &c)
 int tc_dq_buffers(const Problem &p, int bn, int stages)
 {
     const int mode = mode_of(p.op);
-    return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages, packed_group(p, bn, stages));
+    return dq_buffers(is_w4(mode) || mode == kW2A8, bn, stages, packed_group(p, bn, stages), kRowsW,
+                      act_rows(bn, false));
 }
 
 // the deepest activation ring (2..5; 8 for token tiles up to 128, 16 up to 64) that keeps the grouped

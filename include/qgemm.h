@@ -99,10 +99,12 @@ typedef struct qgemm_config_t {
                         runs, so the absolute error grows with |A| (keep |A| < 512)        */
     int32_t bk;      /* TC: tile extent along K                                              */
     int32_t stages;  /* TC: activation ring depth (2..5; 8 for bn <= 128, 16 for bn <= 64;
-                        2..4 when swap_ab = 0)                                               */
+                        2..4 when swap_ab = 0; 2 or 4 half-tile stages when bn = 512)         */
     int32_t split_k; /* number of K parts (1 = no atomics)                                   */
     int32_t swap_ab; /* TC: 1 = weights fill the MMA's M side (bm = 128 weight rows), tokens
-                        its N side (bn = 16..256 tokens); 0 = token-major, W4A16 with a group
+                        its N side (bn = 16..256 tokens, or 512 for packed W4A16 / W2A8:
+                        two 256-token accumulators that share each upcast weight slab, no
+                        double-buffered accumulator); 0 = token-major, W4A16 with a group
                         size that is a multiple of 64: bm = 128 tokens, bn = 256 weight rows
                         (an MMA from shared memory reaches its full rate only at N = 256)    */
 } qgemm_config_t;

@@ -193,10 +193,11 @@ def _tc(bn, stages, split=1):
 
 def test_plan_large_m_uses_tensor_cores():
     c = qg.qgemm_plan(qg.OP_W4A16, 16384, 16384, 16384, 128, 1)
-    assert c["path"] == qg.PATH_TC and c["bn"] == 256 and 2 <= c["stages"] <= 5
-    assert c["split_k"] == 1                     # 8192 tiles fill the GPU many times
-    c = qg.qgemm_plan(qg.OP_W4A16, 16384, 16384, 16384, 128, 1)
+    assert c["path"] == qg.PATH_TC and c["bn"] == 512 and c["stages"] == 4
+    assert c["split_k"] == 1                     # 4096 tiles fill the GPU many times
     assert c["swap_ab"] == 1                     # weights in the MMA's M side
+    c = qg.qgemm_plan(qg.OP_DENSE_F16, 16384, 16384, 16384)
+    assert c["path"] == qg.PATH_TC and c["bn"] == 256 and 2 <= c["stages"] <= 5
     # up to one tile of tokens: the token-major tile (128 tokens x 256 weight rows), K split
     # until the units fill the GPU
     c = qg.qgemm_plan(qg.OP_W4A16, 32, 16384, 16384, 128, 1)
@@ -342,3 +343,41 @@ def test_pair_tile_rules():
     # weights carried in the activation ring (fp16 / int8) leave no room for 8 stages of 256
     with pytest.raises(qg.QGemmError):
         qg.qgemm_set_config(qg.OP_DENSE_F16, 512, 16384, 16384, -1, 0, {**ok, "stages": 8})
+
+
+def test_dual_tile_rules():
+    """512-token weight-major tiles (two 256-token accumulators per upcast slab): packed weights
+    only (W4A16, W2A8, either layout), one CTA, 2 or 4 half-tile activation stages."""
+    ok = {"path": qg.PATH_TC, "rows": 0, "bm": 128, "bn": 512, "bk": 0, "stages": 4,
+          "split_k": 1, "swap_ab": 1}
+    for op, gs in ((qg.OP_W4A16, 128), (qg.OP_W2A8, -1), (qg.OP_W4A16_INTERLEAVED, 128),
+                   (qg.OP_W2A8_INTERLEAVED, -1)):
+        for st in (2, 4):
+            for sk in (1, 3):
+                cfg = {**ok, "stages": st, "split_k": sk}
+                qg.qgemm_set_config(op, 4096, 16384, 16384, gs, 0, cfg)
+                plan = qg.qgemm_plan(op, 4096, 16384, 16384, gs, 0)
+                assert (plan["bn"], plan["stages"], plan["split_k"]) == (512, st, sk)
+                qg.qgemm_set_config(op, 4096, 16384, 16384, gs, 0, None)
+    for bad in ({"stages": 3}, {"stages": 5}, {"bm": 256}, {"swap_ab": 0}):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, 4096, 16384, 16384, 128, 1, {**ok, **bad})
+    for op in (qg.OP_DENSE_F16, qg.OP_W8A8):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(op, 4096, 16384, 16384, -1, 0, ok)
+
+
+def test_dual_tile_default_plan():
+    """The default plan takes the 512-token tile for int4 weights when its schedule of whole
+    waves (a unit of 512 tokens costing 1.71 of 256) is the shorter one, else the 256-token tile."""
+    qg.qgemm_clear_configs()
+    for op in (qg.OP_W4A16, qg.OP_W4A16_INTERLEAVED):
+        for M in (1024, 4096, 16384):
+            c = qg.qgemm_plan(op, M, 16384, 16384, 128, 1)
+            assert (c["path"], c["bn"], c["stages"], c["split_k"]) == (qg.PATH_TC, 512, 4, 1), (M, c)
+    # 3 token tiles of 256 against 2 of 512 on 32 weight tiles: one wave either way
+    c = qg.qgemm_plan(qg.OP_W4A16, 600, 4096, 4096, 128, 1)
+    assert c["bn"] == 256, c
+    # int2 and int8 weights keep the 256-token tile
+    assert qg.qgemm_plan(qg.OP_W2A8, 16384, 16384, 16384, -1, 0)["bn"] == 256
+    assert qg.qgemm_plan(qg.OP_W8A8, 16384, 16384, 16384, -1, 0)["bn"] == 256
