@@ -117,11 +117,12 @@ SWEEP_STAGES = (2, 3, 4, 5)
 
 # DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum),
 # by weight-major token tile: on M = 4096, N = K = 16384 the 256-token tile (3 stages) read
-# 1271.105 MB and wrote 129.454 MB; the 512-token tile (4 half-tile stages) read 816.418 MB and
-# wrote 120.399 MB. An M = 16384 launch runs the same pattern (groups of 2048 tokens against all
-# 128 weight tiles, weights read once per group) 4 times as often, so its traffic is scaled by 4.
+# 1271.105 MB and wrote 129.454 MB; the 512-token tile (4 half-tile stages, transposed 16-byte
+# epilogue stores) read 817.545 MB and wrote 121.407 MB. An M = 16384 launch runs the same
+# pattern (groups of 2048 tokens against all 128 weight tiles, weights read once per group) 4
+# times as often, so its traffic is scaled by 4.
 TRAFFIC_BYTES = {(16384, 16384, 16384, 256): 4 * (1271105000 + 129453568),
-                 (16384, 16384, 16384, 512): 4 * (816417536 + 120399104)}
+                 (16384, 16384, 16384, 512): 4 * (817544704 + 121406976)}
 TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the M = 4096 launch of the "
                   "same tile, scaled by 4 (its 2 groups of 2048 tokens against 8)")
 
