@@ -488,27 +488,35 @@ def run_extras(args, dev, peaks, headline_sps, deadline):
 
 def stage_sweep(op, sp, tuned, peaks):
     """Pipeline depth 2..5 of the tensor-core kernel on this shape, the tuned tile and split
-    kept; each depth timed and parity-checked, then the tuned configuration restored."""
+    kept; each depth timed and parity-checked, then the tuned configuration restored. When the
+    tuned tile is the 512-token one (2 or 4 half-tile stages only), the 256-token tile with the
+    same split is swept over 2..5 as well."""
     import gemv_w4a16_w8a8_b200 as qg
     M, K, N, hz = sp["M"], sp["K"], sp["N"], sp["hz"]
     g_op = GS if op == "w4a16" else -1
     rows = []
     if tuned["path"] != qg.PATH_TC:
         return rows
-    for st in SWEEP_STAGES:
-        cfg = dict(tuned)
-        cfg["stages"] = st
-        try:
-            qg.qgemm_set_config(op_code(op, sp), M, N, K, g_op, hz, cfg)
-        except qg.QGemmError:
-            rows.append({"op": op, "shape_mkn": [M, K, N], "has_zero": hz, "stages": st,
-                         "cfg": cfg, "us": None, "note": "does not fit shared memory"})
-            continue
-        ms = time_shape(op, sp, reps=max(4, min(20, sp["n_sets"])))
-        par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"] + st)
-        r = shape_row(op, sp, ms, cfg, peaks, par)
-        r.update({"op": op, "stages": st})
-        rows.append(r)
+    tiles = [dict(tuned)]
+    if tuned["bn"] == 512:
+        tiles.append(dict(tuned, bn=256))
+    for tile in tiles:
+        for st in SWEEP_STAGES:
+            cfg = dict(tile)
+            cfg["stages"] = st
+            try:
+                qg.qgemm_set_config(op_code(op, sp), M, N, K, g_op, hz, cfg)
+            except qg.QGemmError:
+                note = ("the 512-token tile takes 2 or 4 half-tile stages" if cfg["bn"] == 512
+                        else "does not fit shared memory")
+                rows.append({"op": op, "shape_mkn": [M, K, N], "has_zero": hz, "stages": st,
+                             "cfg": cfg, "us": None, "note": note})
+                continue
+            ms = time_shape(op, sp, reps=max(4, min(20, sp["n_sets"])))
+            par = parity_check(op, sp["h"], sp["C"], M, K, N, hz, sp["seed"] + st)
+            r = shape_row(op, sp, ms, cfg, peaks, par)
+            r.update({"op": op, "stages": st})
+            rows.append(r)
     qg.qgemm_set_config(op_code(op, sp), M, N, K, g_op, hz, tuned)
     return rows
 
