@@ -426,6 +426,7 @@ qgemm_config_t choose(const Problem &p, int split_k, int sms)
     if (split_k > 0) {
         // an explicit split asks for a path that cuts K into exactly that many parts
         if (c.path == QG_PATH_STREAM) c = heuristic(p, sms, false);
+        if (c.path == QG_PATH_TC) c.rows = 0;   // not the stream-K schedule
         c.split_k = split_k;
     }
     return c;
@@ -436,7 +437,7 @@ qgemm_config_t choose(const Problem &p, int split_k, int sms)
 qg_status run(const Problem &p, const qgemm_config_t &c, DeviceInfo *d, cudaStream_t stream)
 {
     if (!supports(p, c)) return QG_ERR_BAD_CONFIG;
-    if (c.split_k > 1 || c.path == QG_PATH_STREAM) {
+    if (c.split_k > 1 || c.path == QG_PATH_STREAM || (c.path == QG_PATH_TC && c.rows == 1)) {
         if (cudaMemsetAsync(p.C, 0, out_bytes(p), stream) != cudaSuccess) {
             cudaGetLastError();
             return QG_ERR_CUDA;
@@ -599,6 +600,19 @@ std::vector<qgemm_config_t> candidates(const Problem &p)
                 if (sk > 1 && tiles >= 2L * kDefaultSms) continue;
                 if (tc_supports(p, t)) out.push_back(t);
             }
+        // the same tile on the stream-K schedule
+        t.stages = 4;
+        t.split_k = 1;
+        t.rows = 1;
+        if (tc_supports(p, t)) out.push_back(t);
+    }
+    if (p.op != QG_OP_DENSE_F16 && p.M > 16) {
+        // stream-K schedule of the default tensor-core tile (every SM an equal share of the work)
+        qgemm_config_t t = (p.op == QG_OP_W4A16 && p.M <= 256) ? tc_toka_default(p, kDefaultSms)
+                                                               : tc_default(p, kDefaultSms);
+        t.split_k = 1;
+        t.rows = 1;
+        if (tc_supports(p, t)) out.push_back(t);
     }
     if (p.op == QG_OP_DENSE_F16 || p.M > 1) {
         const qgemm_config_t base = tc_default(p, kDefaultSms);

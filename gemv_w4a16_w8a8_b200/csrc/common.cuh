@@ -216,6 +216,14 @@ __device__ __forceinline__ void red_add_f16x2(void *p, uint32_t v)
     asm volatile("red.global.add.noftz.f16x2 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// 8 consecutive fp16 values (16-byte aligned)
+__device__ __forceinline__ void red_add_f16x8(void *p, const uint4 &v)
+{
+    asm volatile("red.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void red_add_f16(void *p, uint16_t v)
 {
     asm volatile("red.global.add.noftz.f16 [%0], %1;" ::"l"(p), "h"(v) : "memory");

@@ -366,9 +366,10 @@ __device__ __forceinline__ uint32_t half2_bcast(float x)
 // lanes the token-pair words go through an 8 x 8 transpose (3 shuffle stages: at stage b, lanes
 // whose bit b differs swap the words whose index bit b differs from their own), after which lane
 // i of group g holds tokens 2i and 2i+1 of rows 8g..8g+7 and writes each as one 16-byte store:
-// 2 store instructions per 16 tokens instead of 16 of 4 bytes. Needs N % 8 == 0 and nrow0 % 8 == 0.
+// 2 store instructions per 16 tokens instead of 16 of 4 bytes (with `add`, two 16-byte fp16 atomic
+// adds). Needs N % 8 == 0 and nrow0 % 8 == 0.
 __device__ __forceinline__ void store_rows16(const uint32_t (&v)[16], __half *C, int N, int M,
-                                             int t0, int nrow0, int lane)
+                                             int t0, int nrow0, int lane, bool add)
 {
     uint32_t p[8];
 #pragma unroll
@@ -395,8 +396,14 @@ __device__ __forceinline__ void store_rows16(const uint32_t (&v)[16], __half *C,
                                       prmt_i<0x5410>(p[4], p[5]), prmt_i<0x5410>(p[6], p[7]));
         const uint4 odd = make_uint4(prmt_i<0x7632>(p[0], p[1]), prmt_i<0x7632>(p[2], p[3]),
                                      prmt_i<0x7632>(p[4], p[5]), prmt_i<0x7632>(p[6], p[7]));
-        if (ta < M) *reinterpret_cast<uint4 *>(C + (size_t)ta * N + n) = even;
-        if (ta + 1 < M) *reinterpret_cast<uint4 *>(C + (size_t)(ta + 1) * N + n) = odd;
+        __half *c0 = C + (size_t)ta * N + n;
+        if (add) {
+            if (ta < M) red_add_f16x8(c0, even);
+            if (ta + 1 < M) red_add_f16x8(c0 + N, odd);
+        } else {
+            if (ta < M) *reinterpret_cast<uint4 *>(c0) = even;
+            if (ta + 1 < M) *reinterpret_cast<uint4 *>(c0 + N) = odd;
+        }
     }
 }
 
@@ -405,12 +412,32 @@ struct Unit {
     int n0, t0, kb0, nk;
 };
 
+// kbps > 0: units are (K part of kbps slabs, tile). kbps < 0: stream-K schedule over the grid's G
+// CTAs: the flattened (tile, copy of pg slabs) space is cut into G ranges of equal length, CTA c
+// owning copies [c T / G, (c + 1) T / G); its range crosses at most J = -kbps tiles, and unit
+// u = c + G j is the part of that range in the j-th of them (nk = 0 when there is none).
 __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv, int nkb,
-                                        int kbps, int wr = kRowsW, int group_t = kGroupT)
+                                        int kbps, int wr = kRowsW, int group_t = kGroupT,
+                                        int pg = 1)
 {
     const int tiles = n_tiles * t_tiles;
-    const int split = u / tiles;
-    const int tile = u - split * tiles;
+    int tile, kb0, nk;
+    if (kbps < 0) {
+        const int G = (int)gridDim.x, c = u % G, j = u / G;
+        const int ncp = nkb / pg;
+        const long long T = (long long)tiles * ncp;
+        const long long a = (long long)c * T / G, b = (long long)(c + 1) * T / G;
+        tile = (int)(a / ncp) + j;
+        const long long s0 = max(a, (long long)tile * ncp), s1 = min(b, (long long)(tile + 1) * ncp);
+        if (tile >= tiles || s0 >= s1) return Unit{0, 0, 0, 0};
+        kb0 = (int)(s0 - (long long)tile * ncp) * pg;
+        nk = (int)(s1 - s0) * pg;
+    } else {
+        const int split = u / tiles;
+        tile = u - split * tiles;
+        kb0 = split * kbps;
+        nk = max(0, min(nkb, kb0 + kbps) - kb0);
+    }
     const int per_group = group_t * n_tiles;
     const int group = tile / per_group;
     const int first_t = group * group_t;
@@ -419,8 +446,8 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
     Unit w;
     w.t0 = (first_t + within % gt) * BNv;
     w.n0 = (within / gt) * wr;
-    w.kb0 = split * kbps;
-    w.nk = max(0, min(nkb, w.kb0 + kbps) - w.kb0);
+    w.kb0 = kb0;
+    w.nk = nk;
     return w;
 }
 
@@ -559,7 +586,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         int it = 0;
         bool stop = false;
         for (int u = ustart; u < units && !stop; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
             for (int i = 0; i < NH * w.nk; ++i, ++it) {
                 const int s = it % STAGES;
                 if (!warp_wait(empty_bar(s), ((it / STAGES) & 1) ^ 1, abort_flag, err)) {
@@ -609,7 +636,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             int it = 0;
             bool stop = false;
             for (int u = ustart; u < units && !stop; u += ustep) {
-                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+                const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
                 // units cover whole copies: with PG > 1 the split and K are multiples of PG slabs
                 for (int i = 0; i < w.nk; i += PG, ++it) {
                     const int p = it % SP;
@@ -636,7 +663,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         int it = 0, sa = 0, j = 0;   // slabs, activation stages and units consumed
         bool stop = false;
         for (int u = ustart; u < units && !stop; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
             if (w.nk == 0) continue;
             const int b = NBUF == 2 ? j & 1 : 0;
             const int use = NBUF == 2 ? j >> 1 : j;     // earlier uses of buffer b
@@ -742,10 +769,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 while (c.u < units && c.i >= c.w.nk) {
                     c.u += ustep;
                     c.i = 0;
-                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+                    if (c.u < units) c.w = unit_of(c.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
                 }
             };
-            Cursor cur{ustart, 0, unit_of(ustart, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT)};
+            Cursor cur{ustart, 0, unit_of(ustart, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG)};
             settle(cur);
             // Scales and zeros. Per slab a thread needs s[n][g] and z[n][g] of its row n. Loading
             // those 2-byte values one slab at a time makes every warp touch 32 rows (32 sectors)
@@ -777,7 +804,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             };
             // the window after wnd in this CTA's walk (same unit, or the next unit's first one)
             auto next_window = [&](Window &out, const Window &wnd) {
-                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+                const Unit w = unit_of(wnd.u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
                 const int g_last = min(((w.kb0 + w.nk) * 64 - 1) / gs, G - 1);
                 if (wnd.gb + 8 <= g_last) {
                     load_window(out, wnd.u, w, wnd.gb + 8);
@@ -786,7 +813,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 int u = wnd.u + ustep;
                 Unit nw = w;
                 while (u < units) {
-                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+                    nw = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
                     if (nw.nk > 0) break;
                     u += ustep;
                 }
@@ -965,7 +992,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         const bool pairs = (N & 1) == 0;
         int j = 0;
         for (int u = ustart; u < units; u += ustep) {
-            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT);
+            const Unit w = unit_of(u, n_tiles, t_tiles, BN, nkb, kb_per_split, UR, GT, PG);
             if (w.nk == 0) continue;
             const int b = NBUF == 2 ? j & 1 : 0;
             bool ok = mbar_wait(accf_bar(b), (NBUF == 2 ? j >> 1 : j) & 1, abort_flag, err);
@@ -995,7 +1022,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                             h2[i] = pack_half2_rn(__uint_as_float(v[2 * i]),
                                                   __uint_as_float(v[2 * i + 1]));
                         if (n + 16 <= N && pairs) {
-                            if (atomic_out) {
+                            if (atomic_out && vec16) {
+                                red_add_f16x8(dst, make_uint4(h2[0], h2[1], h2[2], h2[3]));
+                                red_add_f16x8(dst + 8, make_uint4(h2[4], h2[5], h2[6], h2[7]));
+                            } else if (atomic_out) {
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) red_add_f16x2(dst + 2 * i, h2[i]);
                             } else if (vec16) {
@@ -1018,8 +1048,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                 }
             } else {
                 const int n = w.n0 + roff + r;
-                // fp16 results without atomics leave as 16-byte stores of 8 rows
-                const bool rows16 = !atomic_out && (N & 7) == 0;
+                // fp16 results leave as 16-byte stores (or 16-byte atomic adds) of 8 rows
+                const bool rows16 = (N & 7) == 0;
                 // int8 requantisation (int32 modes): this lane's output-channel multiplier
                 const float rq = (T::c_bytes == 4 && mult && n < N) ? mult[n] : 0.f;
                 const uint32_t lane_addr =
@@ -1032,7 +1062,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     if constexpr (T::c_bytes == 2) {
                         if (rows16) {
                             store_rows16(v, static_cast<__half *>(C), N, M, w.t0 + c,
-                                         w.n0 + roff + 32 * warp, lane);
+                                         w.n0 + roff + 32 * warp, lane, atomic_out != 0);
                             continue;
                         }
                     }
@@ -1125,8 +1155,11 @@ int packed_group(const Problem &p, int bn, int stages, int wr = kRowsW, bool pai
     return smem_bytes(mode, bn, stages, 4, wr, pair) <= kMaxSmem ? 4 : 1;
 }
 
+// streamk: the stream-K schedule (every CTA gets an equal share of the (tile, K) work; partial
+// tiles are added into the zeroed output)
 template <int MODE, int BN, int STAGES, int PG, bool TOKA = false, bool PAIR = false>
-cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream)
+cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStream_t stream,
+                     bool streamk = false)
 {
     using T = Traits<MODE>;
     using L = Smem<MODE, BN, STAGES, PG, TOKA, PAIR>;
@@ -1178,8 +1211,9 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
     constexpr int UR = PAIR ? 2 * kRowsW : L::WR;      // weight rows per unit
     const int n_tiles = (p.N + UR - 1) / UR;
     const int t_tiles = (p.M + BN - 1) / BN;
-    const long units = (long)n_tiles * t_tiles * splits;
+    long units = (long)n_tiles * t_tiles * splits;
     if (units > 0x7fffffffL) return cudaErrorInvalidValue;
+    if (streamk && (PAIR || nkb % PG)) return cudaErrorInvalidValue;
     // persistent grid: as many CTAs (CTA pairs) as fit on the device at once (shared memory,
     // threads and the TMEM columns each CTA holds), never more than there are units
     static int per_dev[64] = {};
@@ -1216,12 +1250,21 @@ cudaError_t launch_t(const Problem &p, int split_k, unsigned int *err, cudaStrea
         if (resident <= 0) return cudaErrorInvalidConfiguration;
         per_dev[dev] = resident;
     }
+    int kb_arg = kbps;
+    if (streamk) {
+        // G CTAs, each owning ceil(T / G) copies at most, which cross at most J tiles
+        const long G = per_dev[dev], ncp = nkb / PG, T = (long)n_tiles * t_tiles * ncp;
+        const long J = ((T + G - 1) / G + ncp - 1) / ncp + 1;
+        units = G * J;
+        if (units > 0x7fffffffL) return cudaErrorInvalidValue;
+        kb_arg = -(int)J;
+    }
     const int slots = (int)std::min<long>(units, (long)per_dev[dev]);
     cfg.gridDim = dim3(PAIR ? 2 * slots : slots);
     const cudaError_t e = cudaLaunchKernelEx(
         &cfg, kern, tw, ta, static_cast<const __half *>(p.scales),
         p.has_zero ? static_cast<const __half *>(p.zeros) : nullptr, p.C, p.M, p.N, p.K, p.gs,
-        kbps, (int)units, split_k > 1 ? 1 : 0, p.mult, err);
+        kb_arg, (int)units, (split_k > 1 || streamk) ? 1 : 0, p.mult, err);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1231,18 +1274,18 @@ cudaError_t launch_stages_pg(const Problem &p, const qgemm_config_t &c, unsigned
                              cudaStream_t stream)
 {
     switch (c.stages) {
-    case 2: return launch_t<MODE, BN, 2, PG>(p, c.split_k, err, stream);
-    case 3: return launch_t<MODE, BN, 3, PG>(p, c.split_k, err, stream);
-    case 4: return launch_t<MODE, BN, 4, PG>(p, c.split_k, err, stream);
-    case 5: return launch_t<MODE, BN, 5, PG>(p, c.split_k, err, stream);
+    case 2: return launch_t<MODE, BN, 2, PG>(p, c.split_k, err, stream, c.rows == 1);
+    case 3: return launch_t<MODE, BN, 3, PG>(p, c.split_k, err, stream, c.rows == 1);
+    case 4: return launch_t<MODE, BN, 4, PG>(p, c.split_k, err, stream, c.rows == 1);
+    case 5: return launch_t<MODE, BN, 5, PG>(p, c.split_k, err, stream, c.rows == 1);
     default: break;
     }
     // deep activation rings for small token tiles: a small activation copy waits ~2-3 us behind
     // the weight stream, so only many stages in flight keep the MMA fed
     if constexpr (BN <= 128)
-        if (c.stages == 8) return launch_t<MODE, BN, 8, PG>(p, c.split_k, err, stream);
+        if (c.stages == 8) return launch_t<MODE, BN, 8, PG>(p, c.split_k, err, stream, c.rows == 1);
     if constexpr (BN <= 64)
-        if (c.stages == 16) return launch_t<MODE, BN, 16, PG>(p, c.split_k, err, stream);
+        if (c.stages == 16) return launch_t<MODE, BN, 16, PG>(p, c.split_k, err, stream, c.rows == 1);
     return cudaErrorInvalidValue;
 }
 
@@ -1262,12 +1305,12 @@ cudaError_t launch_toka(const Problem &p, const qgemm_config_t &c, unsigned int 
 {
     const bool g4 = packed_group(p, kTokT, c.stages, kRowsT) == 4;
     switch (c.stages) {
-    case 2: return g4 ? launch_t<MODE, kTokT, 2, 4, true>(p, c.split_k, err, stream)
-                      : launch_t<MODE, kTokT, 2, 1, true>(p, c.split_k, err, stream);
-    case 3: return g4 ? launch_t<MODE, kTokT, 3, 4, true>(p, c.split_k, err, stream)
-                      : launch_t<MODE, kTokT, 3, 1, true>(p, c.split_k, err, stream);
-    case 4: return g4 ? launch_t<MODE, kTokT, 4, 4, true>(p, c.split_k, err, stream)
-                      : launch_t<MODE, kTokT, 4, 1, true>(p, c.split_k, err, stream);
+    case 2: return g4 ? launch_t<MODE, kTokT, 2, 4, true>(p, c.split_k, err, stream, c.rows == 1)
+                      : launch_t<MODE, kTokT, 2, 1, true>(p, c.split_k, err, stream, c.rows == 1);
+    case 3: return g4 ? launch_t<MODE, kTokT, 3, 4, true>(p, c.split_k, err, stream, c.rows == 1)
+                      : launch_t<MODE, kTokT, 3, 1, true>(p, c.split_k, err, stream, c.rows == 1);
+    case 4: return g4 ? launch_t<MODE, kTokT, 4, 4, true>(p, c.split_k, err, stream, c.rows == 1)
+                      : launch_t<MODE, kTokT, 4, 1, true>(p, c.split_k, err, stream, c.rows == 1);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -1297,10 +1340,10 @@ cudaError_t launch_dual(const Problem &p, const qgemm_config_t &c, unsigned int 
     if constexpr (is_w4(MODE) || is_w2(MODE)) {
         const bool g4 = packed_group(p, 512, c.stages) == 4;
         switch (c.stages) {
-        case 2: return g4 ? launch_t<MODE, 512, 2, 4>(p, c.split_k, err, stream)
-                          : launch_t<MODE, 512, 2, 1>(p, c.split_k, err, stream);
-        case 4: return g4 ? launch_t<MODE, 512, 4, 4>(p, c.split_k, err, stream)
-                          : launch_t<MODE, 512, 4, 1>(p, c.split_k, err, stream);
+        case 2: return g4 ? launch_t<MODE, 512, 2, 4>(p, c.split_k, err, stream, c.rows == 1)
+                          : launch_t<MODE, 512, 2, 1>(p, c.split_k, err, stream, c.rows == 1);
+        case 4: return g4 ? launch_t<MODE, 512, 4, 4>(p, c.split_k, err, stream, c.rows == 1)
+                          : launch_t<MODE, 512, 4, 1>(p, c.split_k, err, stream, c.rows == 1);
         default: break;
         }
     }
@@ -1332,6 +1375,10 @@ cudaError_t launch_bn(const Problem &p, const qgemm_config_t &c, unsigned int *e
 bool tc_supports(const Problem &p, const qgemm_config_t &c)
 {
     if (c.path != QG_PATH_TC) return false;
+    // rows = 1: the stream-K schedule (single-CTA tiles, results added into the zeroed output:
+    // not for the requantised int8 output, which needs whole sums)
+    if (c.rows != 0 && c.rows != 1) return false;
+    if (c.rows == 1 && (c.bm == 2 * kRowsW || c.split_k != 1 || p.mult)) return false;
     if (!c.swap_ab) {
         // token-major variant: W4A16 with scale groups of whole slabs
         if (p.op != QG_OP_W4A16 || c.bm != kTokT || c.bn != kRowsT) return false;

@@ -87,7 +87,12 @@ typedef enum qg_path {
 /* One launch configuration. Fields a path does not use are ignored (set them to 0). */
 typedef struct qgemm_config_t {
     int32_t path;    /* qg_path                                                             */
-    int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise)  */
+    int32_t rows;    /* GEMV: weight rows per warp (16, 32 or 64 for W4A16; 1..8 otherwise).
+                        TC (one CTA per tile, split_k = 1): 1 = stream-K schedule: the
+                        (tile, K) work is cut into one equal share per persistent CTA and
+                        partial tiles are added into the zeroed output (fp16 / int32 atomics,
+                        so fp16 results can differ in the last bits from run to run); not for
+                        qgemm_w8a8_requant. 0 = one whole tile (or K part) per work unit.   */
     int32_t bm;      /* TC: tile extent along the MMA's M: 128 (one CTA), or 256 for the
                         weight-major tile shared by a CTA pair (one cta_group::2 MMA over
                         two SMs: 256 weight rows, bn = 128 or 256 tokens, stages 3, 4, 5 or 8) */

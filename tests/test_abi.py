@@ -381,3 +381,21 @@ def test_dual_tile_default_plan():
     # int2 and int8 weights keep the 256-token tile
     assert qg.qgemm_plan(qg.OP_W2A8, 16384, 16384, 16384, -1, 0)["bn"] == 256
     assert qg.qgemm_plan(qg.OP_W8A8, 16384, 16384, 16384, -1, 0)["bn"] == 256
+
+
+def test_stream_k_schedule_rules():
+    """rows = 1 on a tensor-core config selects the stream-K schedule: single-CTA tiles (either
+    orientation, any token tile), split_k = 1; the CTA pair and other rows values are refused."""
+    base = {"path": qg.PATH_TC, "rows": 1, "bm": 128, "bn": 256, "bk": 0, "stages": 3,
+            "split_k": 1, "swap_ab": 1}
+    cases = [(qg.OP_W4A16, 128, base), (qg.OP_W4A16, 128, {**base, "bn": 512, "stages": 4}),
+             (qg.OP_W4A16, 128, {**base, "swap_ab": 0, "stages": 3}),
+             (qg.OP_W2A8, -1, base), (qg.OP_W8A8, -1, base), (qg.OP_DENSE_F16, -1, {**base, "stages": 4})]
+    for op, gs, cfg in cases:
+        M = 128 if cfg["swap_ab"] == 0 else 512
+        qg.qgemm_set_config(op, M, 16384, 16384, gs, 0, cfg)
+        assert qg.qgemm_plan(op, M, 16384, 16384, gs, 0)["rows"] == 1
+        qg.qgemm_set_config(op, M, 16384, 16384, gs, 0, None)
+    for bad in ({"split_k": 2}, {"rows": 2}, {"bm": 256}):
+        with pytest.raises(qg.QGemmError):
+            qg.qgemm_set_config(qg.OP_W4A16, 512, 16384, 16384, 128, 1, {**base, **bad})
