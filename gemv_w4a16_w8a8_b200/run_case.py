@@ -45,6 +45,7 @@ def main(argv=None) -> int:
 
     dev = torch.device("cuda", 0)
     M, N, K = a.M, a.N, a.K
+    ks = [a.split_k]
     up = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(dev)
     opc = {"w4a16": qg.OP_W4A16, "w8a8": qg.OP_W8A8, "w2a8": qg.OP_W2A8,
            "dense": qg.OP_DENSE_F16}[a.op]
@@ -61,14 +62,14 @@ def main(argv=None) -> int:
         S = up(d["scales"])
         Z = up(d["zeros"]) if hz else None
         wbytes = N * K // 2
-        run = lambda w, C: mm(A, w, S, Z, C=C, group_size=gs, split_k=a.split_k)
+        run = lambda w, C: mm(A, w, S, Z, C=C, group_size=gs, split_k=ks[0])
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + N * (K // (K if gs <= 0 else gs)) * 2 * (1 + hz) + 2 * M * K + 2 * M * N
     elif a.op == "w8a8":
         d = synth.w8a8_inputs(M, N, K, seed=0)
         A, W = up(d["A"]), up(d["W"])
         wbytes = N * K
-        run = lambda w, C: qg.qgemm_w8a8(A, w, C=C, split_k=a.split_k)
+        run = lambda w, C: qg.qgemm_w8a8(A, w, C=C, split_k=ks[0])
         C = torch.empty((M, N), dtype=torch.int32, device=dev)
         nbytes = wbytes + M * K + 4 * M * N
     elif a.op == "w2a8":
@@ -77,18 +78,22 @@ def main(argv=None) -> int:
         mm = qg.qgemm_w2a8_interleaved if ilv else qg.qgemm_w2a8
         A, W = up(d["A"]), pack(up(d["Wv"]))
         wbytes = N * K // 4
-        run = lambda w, C: mm(A, w, C=C, split_k=a.split_k)
+        run = lambda w, C: mm(A, w, C=C, split_k=ks[0])
         C = torch.empty((M, N), dtype=torch.int32, device=dev)
         nbytes = wbytes + M * K + 4 * M * N
     else:
         d = synth.dense_inputs(M, N, K, seed=0)
         A, W = up(d["A"]), up(d["W"])
         wbytes = 2 * N * K
-        run = lambda w, C: qg.qgemm_dense_f16(A, w, C=C, split_k=a.split_k)
+        run = lambda w, C: qg.qgemm_dense_f16(A, w, C=C, split_k=ks[0])
         C = torch.empty((M, N), dtype=torch.float16, device=dev)
         nbytes = wbytes + 2 * M * K + 2 * M * N
 
+    # the call's own split_k: 0 (the plan) once a configuration is pinned below, so that the
+    # pinned one runs as given (an explicit split would override its schedule)
+    ks[0] = a.split_k
     if a.path or a.rows or a.bn or a.bk or a.bm or a.stages >= 0 or a.swap_ab >= 0:
+        ks[0] = 0
         cfg = qg.qgemm_plan(opc, M, N, K, gs, hz)
         if a.path and a.path != cfg["path"]:
             cfg = {k: 0 for k in cfg}
@@ -102,7 +107,7 @@ def main(argv=None) -> int:
         if a.swap_ab >= 0:
             cfg["swap_ab"] = a.swap_ab
         qg.qgemm_set_config(opc, M, N, K, gs, hz, cfg)
-    print("config", qg.qgemm_plan(opc, M, N, K, gs, hz, a.split_k))
+    print("config", qg.qgemm_plan(opc, M, N, K, gs, hz, ks[0]))
 
     copies = a.copies or max(1, min(64, math.ceil(3 * 126 * 2 ** 20 / wbytes)))
     Ws = [W] + [W.clone() for _ in range(copies - 1)]
@@ -123,7 +128,7 @@ def main(argv=None) -> int:
     qg.qgemm_sync_check()
     us = e0.elapsed_time(e1) * 1e3 / a.iters
     flops = 2.0 * M * N * K
-    cfg_used = qg.qgemm_plan(opc, M, N, K, gs, hz, a.split_k)
+    cfg_used = qg.qgemm_plan(opc, M, N, K, gs, hz, ks[0])
     print(f"{a.op} M={M} N={N} K={K}: {us:.2f} us/call  {nbytes / us / 1e3:.1f} GB/s  "
           f"{flops / us / 1e6:.2f} TFLOP/s  ({copies} weight copies)  cfg={cfg_used}")
     qg.qgemm_set_config(opc, M, N, K, gs, hz, None)
