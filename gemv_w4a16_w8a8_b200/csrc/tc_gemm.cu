@@ -5,7 +5,9 @@
 // Two tile orientations, because an MMA from shared memory at M = 128 occupies the tensor pipe
 // ~98 cycles for any N up to 128 and reaches its full rate only at N = 256 (measured):
 //   weight-major   D[128 weight rows, BN tokens] = W_tile . A_tile^T, BN in {16..256}; the
-//                  large-M tile (BN = 256) upcasts each weight once per 256 tokens;
+//                  large-M tile (BN = 256) upcasts each weight once per 256 tokens, and the
+//                  512-token tile of the packed formats feeds each upcast slab to two N = 256
+//                  MMAs (two accumulators filling TMEM), once per 512 tokens;
 //   token-major    D[128 tokens, 256 weight rows] = A_tile . W_tile^T (W4A16): tokens are the A
 //                  operand (rows past M read as zero), 256 upcast weight rows the B operand, so
 //                  every MMA runs at N = 256 for 1..128 tokens.
@@ -22,8 +24,11 @@
 //   warps 8-15  upcast of packed weights into the K-major SWIZZLE_128B layout the MMA reads
 //               (LOP3 magic-number upcast, PRMT re-ordering, HFMA2 with the group's scale and
 //               zero), handed over per slab or per copy;
-//   warps 0-3   epilogue: tcgen05.ld of the double-buffered accumulator, conversion, stores or
-//               red.global.add for split-K (parallel-k through atomics, hidet issue #364).
+//   warps 0-3   epilogue: tcgen05.ld of the (double-buffered) accumulator, conversion, stores or
+//               red.global.add for split-K and stream-K (parallel-k through atomics, hidet issue
+//               #364); weight-major fp16 results leave as 16-byte rows after a shuffle transpose.
+// Work units: whole tiles, K parts of them (split-K), or equal shares of the flattened (tile, K)
+// work per persistent CTA (stream-K).
 // Every wait is bounded (%globaltimer); a wait that runs out raises the device error word, makes
 // the other roles stop, lets in-flight copies land, frees TMEM and returns.
 #include <cuda.h>
@@ -453,7 +458,8 @@ __device__ __forceinline__ Unit unit_of(int u, int n_tiles, int t_tiles, int BNv
 
 // Persistent kernel: each CTA walks work units blockIdx.x, blockIdx.x + gridDim.x, ... The
 // shared-memory ring runs on across units, and the accumulator is double-buffered in TMEM so the
-// epilogue of one unit overlaps the main loop of the next.
+// epilogue of one unit overlaps the main loop of the next (except in the 512-token tile, whose
+// two accumulators fill TMEM: there the next unit's MMAs wait for the epilogue).
 //   warps 0-3  epilogue (warp w reads TMEM lanes 32w..32w+31)
 //   warp 4     TMA producer          warp 5  TMEM allocation + MMA issue
 //   warp 6     TMA producer of packed weight slabs (packed formats)
